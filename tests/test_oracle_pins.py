@@ -1,0 +1,369 @@
+"""Pins for the CPU oracle: what the pages and plain mathematics fix.
+
+None of these re-types the oracle's own formula: each compares it with a
+closed form, a value the pages print (``tests/golden``), brute force on tiny
+inputs written independently here, or a special case that reduces to a
+dense FFN.  Each test names the mistake it would catch.
+"""
+import itertools
+import json
+import math
+import pathlib
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = pathlib.Path(__file__).parent / "golden"
+MODES = (oracle.SOFTMAX_ALL_RENORM, oracle.SOFTMAX_TOPK, oracle.SIGMOID_TOPK_RENORM)
+
+
+def _rand(rng, *shape, scale=1.0):
+    return rng.standard_normal(shape) * scale
+
+
+def _layer(rng, T=9, d=6, E=5, f=4):
+    x = _rand(rng, T, d)
+    wr = _rand(rng, E, d, scale=0.7)
+    wgu = _rand(rng, E, 2 * f, d, scale=0.5)
+    wd = _rand(rng, E, d, f, scale=0.5)
+    return x, wr, wgu, wd
+
+
+def _experts(wgu, wd):
+    f = wd.shape[2]
+    return lambda e: (wgu[e, :f], wgu[e, f:], wd[e])
+
+
+# ------------------------------------------------------------------ pure-Python references
+def _dot(a, b):
+    return math.fsum(p * q for p, q in zip(a, b))
+
+
+def _swiglu_loops(xv, wg, wu, wd):
+    """Dense SwiGLU FFN of one token with explicit loops (independent of numpy @)."""
+    f = len(wg)
+    h = []
+    for j in range(f):
+        g = _dot(xv, wg[j])
+        u = _dot(xv, wu[j])
+        h.append(g / (1.0 + math.exp(-g)) * u)
+    return [_dot(h, wd[i]) for i in range(len(wd))]
+
+
+# ------------------------------------------------------------------ scores and weights
+@pytest.mark.parametrize("E", [1, 2, 8, 256])
+def test_softmax_sums_to_one(E):
+    rng = np.random.default_rng(E)
+    p = oracle.softmax(_rand(rng, 64, E, scale=4.0), axis=1)
+    assert np.all(p > 0)
+    assert np.max(np.abs(p.sum(axis=1) - 1.0)) <= 1e-12
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("E,k", [(8, 1), (8, 2), (128, 4), (256, 8), (6, 6)])
+def test_routing_weights_sum_to_one_and_positive(mode, E, k):
+    rng = np.random.default_rng(10 * E + k)
+    x = _rand(rng, 50, 16)
+    wr = _rand(rng, E, 16, scale=0.5)
+    bias = _rand(rng, E, scale=0.3)
+    r = oracle.route(x, wr, bias, k, mode, bias_select_only=1)
+    assert np.all(r.w > 0)
+    assert np.max(np.abs(r.w.sum(axis=1) - 1.0)) <= 1e-12
+
+
+def test_k1_renormalised_weight_is_one():
+    """[SEV] "Why top-1 routing cannot renormalise": with k=1 the weight is exactly 1."""
+    rng = np.random.default_rng(1)
+    x = _rand(rng, 40, 12)
+    wr = _rand(rng, 8, 12)
+    for mode in MODES:
+        r = oracle.route(x, wr, None, 1, mode)
+        assert np.all(r.w == 1.0)
+
+
+def test_softmax_before_and_after_topk_agree():
+    """[SEV] "Softmax before or after the top-k step": renormalised full
+    softmax equals softmax over the kept logits: the common denominator
+    cancels.  The page measured a difference under 1e-7 on 512 tokens in
+    float32; in float64 only rounding remains."""
+    rng = np.random.default_rng(2)
+    x = _rand(rng, 512, 64)
+    wr = _rand(rng, 8, 64, scale=0.125)
+    a = oracle.route(x, wr, None, 2, oracle.SOFTMAX_ALL_RENORM)
+    b = oracle.route(x, wr, None, 2, oracle.SOFTMAX_TOPK)
+    assert np.array_equal(a.ids, b.ids)
+    assert np.max(np.abs(a.w - b.w)) <= 1e-12
+
+
+def test_topk_matches_brute_force_sort_and_repeated_argmax():
+    """Selection vs a pure-Python sort of (key desc, index asc) pairs and k rounds of argmax.
+    Catches an ascending sort, a wrong tie rule or a dropped slot."""
+    rng = np.random.default_rng(3)
+    key = np.round(_rand(rng, 200, 10), 1)   # coarse values force many exact ties
+    for k in (1, 2, 3, 10):
+        ids = oracle.topk_select(key, k)
+        for t in range(key.shape[0]):
+            brute = [e for _, e in sorted((-key[t, e], e) for e in range(10))][:k]
+            assert ids[t].tolist() == brute
+            rest = list(range(10))
+            picks = []
+            for _ in range(k):
+                best = rest[0]
+                for e in rest[1:]:
+                    if key[t, e] > key[t, best]:
+                        best = e
+                picks.append(best)
+                rest.remove(best)
+            assert ids[t].tolist() == picks
+
+
+def test_topk_gap_brute_force():
+    rng = np.random.default_rng(4)
+    key = _rand(rng, 30, 7)
+    gap = oracle.topk_gap(key, 3)
+    for t in range(30):
+        s = sorted(key[t].tolist(), reverse=True)
+        assert gap[t] == pytest.approx(s[2] - s[3], abs=0)
+    assert np.all(np.isinf(oracle.topk_gap(key, 7)))
+
+
+def test_softmax_topk_is_shift_invariant_sigmoid_is_not():
+    """Softmax weights ignore a constant added to every logit; sigmoid weights do not
+    (catches a sigmoid rule that silently used softmax, or the reverse)."""
+    rng = np.random.default_rng(5)
+    x = _rand(rng, 20, 8)
+    wr = _rand(rng, 6, 8)
+    shift = np.full(6, 0.75)
+    for mode in (oracle.SOFTMAX_ALL_RENORM, oracle.SOFTMAX_TOPK):
+        a = oracle.route(x, wr, None, 3, mode)
+        b = oracle.route(x, wr, shift, 3, mode)
+        assert np.array_equal(a.ids, b.ids)
+        assert np.allclose(a.w, b.w, rtol=0, atol=1e-14)
+    a = oracle.route(x, wr, None, 3, oracle.SIGMOID_TOPK_RENORM)
+    b = oracle.route(x, wr, shift, 3, oracle.SIGMOID_TOPK_RENORM, bias_select_only=0)
+    assert np.array_equal(a.ids, b.ids)
+    assert np.max(np.abs(a.w - b.w)) > 1e-3
+
+
+def test_sigmoid_bias_steers_selection_only():
+    """[AFD] "Why load balancing is the hard part of MoE": the bias shifts routing
+    without distorting the gate values used for output."""
+    rng = np.random.default_rng(6)
+    x = _rand(rng, 64, 16)
+    wr = _rand(rng, 16, 16, scale=0.25)
+    bias = _rand(rng, 16, scale=2.0)
+    r = oracle.route(x, wr, bias, 4, oracle.SIGMOID_TOPK_RENORM, bias_select_only=1)
+    # hand computation of the weights from the unbiased logits on the chosen ids
+    for t in range(64):
+        g = [1.0 / (1.0 + math.exp(-_dot(x[t], wr[e]))) for e in r.ids[t]]
+        assert r.w[t].tolist() == pytest.approx([v / sum(g) for v in g], rel=1e-13)
+    # and the selection did follow the biased key
+    keys = x @ wr.T + bias
+    assert np.array_equal(r.ids, oracle.topk_select(keys, 4))
+
+
+def test_huge_bias_forces_an_expert_and_zero_bias_is_no_bias():
+    rng = np.random.default_rng(7)
+    x = _rand(rng, 33, 8)
+    wr = _rand(rng, 5, 8)
+    bias = np.zeros(5)
+    bias[3] = 1e6
+    for mode in MODES:
+        r = oracle.route(x, wr, bias, 2, mode, bias_select_only=1)
+        assert np.all(r.ids[:, 0] == 3)
+        a = oracle.route(x, wr, None, 2, mode)
+        b = oracle.route(x, wr, np.zeros(5), 2, mode)
+        assert np.array_equal(a.ids, b.ids) and np.array_equal(a.w, b.w)
+
+
+# ------------------------------------------------------------------ dispatch
+@pytest.mark.parametrize("T,E,k", [(1, 1, 1), (17, 4, 2), (100, 8, 2), (64, 256, 8), (5, 6, 6)])
+def test_dispatch_is_a_stable_grouping(T, E, k):
+    rng = np.random.default_rng(T * 31 + E)
+    key = _rand(rng, T, E)
+    ids = oracle.topk_select(key, k)
+    counts, offsets, perm, row_of = oracle.dispatch(ids, E)
+    assert counts.sum() == T * k and offsets[0] == 0 and offsets[E] == T * k
+    assert np.array_equal(np.diff(offsets), counts)
+    assert np.array_equal(np.sort(perm), np.arange(T * k))          # bijection
+    assert np.array_equal(row_of[perm], np.arange(T * k))           # inverse
+    # brute force: rows are the (expert, token, slot) triples in lexicographic order
+    triples = sorted((int(ids[t, s]), t, s) for t in range(T) for s in range(k))
+    assert perm.tolist() == [t * k + s for _, t, s in triples]
+    for e in range(E):
+        assert counts[e] == sum(1 for tr in triples if tr[0] == e)
+
+
+def test_toy_run_tokens_per_expert_sum():
+    """[SEV] build: the tokens-per-expert list adds up to 512 tokens x 2 picks."""
+    g = json.loads((GOLDEN / "param_counts.json").read_text())["toy_layer"]
+    rng = np.random.default_rng(0)
+    x = _rand(rng, g["tokens"], g["d_model"])
+    wr = _rand(rng, g["n_experts"], g["d_model"], scale=0.125)
+    r = oracle.route(x, wr, None, g["top_k"], oracle.SOFTMAX_ALL_RENORM)
+    counts, *_ = oracle.dispatch(r.ids, g["n_experts"])
+    assert int(counts.sum()) == g["tokens_per_expert_sum"]
+
+
+# ------------------------------------------------------------------ expert FFN and layer
+def test_swiglu_closed_form_fixes_gate_up_order():
+    """d = f = 1: y = Wd * SiLU(Wg x) * (Wu x) = -1.5 * SiLU(1) * 6.
+    Swapping gate and up would give -1.5 * SiLU(6) * 1 instead."""
+    y = oracle.swiglu_expert(np.array([[2.0]]), np.array([[0.5]]), np.array([[3.0]]), np.array([[-1.5]]))
+    silu1 = 1.0 / (1.0 + math.exp(-1.0))
+    assert y[0, 0] == pytest.approx(-9.0 * silu1, rel=1e-15)
+    assert abs(y[0, 0] - (-1.5 * 6.0 / (1.0 + math.exp(-6.0)))) > 1.0
+
+
+def test_silu_and_sigmoid_special_values():
+    assert oracle.silu(np.array([0.0]))[0] == 0.0
+    assert oracle.sigmoid(np.array([0.0]))[0] == 0.5
+    assert oracle.silu(np.array([40.0]))[0] == pytest.approx(40.0, rel=1e-15)
+    assert abs(oracle.silu(np.array([-800.0]))[0]) == 0.0
+    assert oracle.silu(np.array([1.0]))[0] == pytest.approx(0.7310585786300049, rel=1e-15)
+
+
+def test_single_expert_layer_is_a_dense_ffn():
+    """E = 1, k = 1 (k = E with one expert): the layer is the dense SwiGLU FFN."""
+    rng = np.random.default_rng(8)
+    x, wr, wgu, wd = _layer(rng, T=7, d=5, E=1, f=3)
+    for mode in MODES:
+        y, r, _ = oracle.moe_layer(x, wr, None, 1, mode, _experts(wgu, wd), 1)
+        for t in range(7):
+            ref = _swiglu_loops(x[t], wgu[0, :3], wgu[0, 3:], wd[0])
+            assert y[t].tolist() == pytest.approx(ref, rel=1e-12, abs=1e-13)
+
+
+def _dense_with_zero_weights(x, wr, bias, k, mode, wgu, wd, bias_select_only=0):
+    """[SEV] build: "a slow version that runs every expert with zero weights for
+    unpicked ones" -- written here with loops over tokens and all experts."""
+    T, d = x.shape
+    E = wr.shape[0]
+    f = wd.shape[2]
+    y = np.zeros_like(x)
+    for t in range(T):
+        logits = [_dot(x[t], wr[e]) for e in range(E)]
+        key = [logits[e] + (0.0 if bias is None else bias[e]) for e in range(E)]
+        chosen = [e for _, e in sorted((-key[e], e) for e in range(E))][:k]
+        if mode == oracle.SOFTMAX_ALL_RENORM:
+            m = max(key)
+            p = [math.exp(v - m) for v in key]
+            z = sum(p)
+            p = [v / z for v in p]
+            s = sum(p[e] for e in chosen)
+            weight = {e: p[e] / s for e in chosen}
+        elif mode == oracle.SOFTMAX_TOPK:
+            m = max(key[e] for e in chosen)
+            ex = {e: math.exp(key[e] - m) for e in chosen}
+            s = sum(ex.values())
+            weight = {e: ex[e] / s for e in chosen}
+        else:
+            sc = logits if bias_select_only else key
+            g = {e: 1.0 / (1.0 + math.exp(-sc[e])) for e in chosen}
+            s = sum(g.values())
+            weight = {e: g[e] / s for e in chosen}
+        for e in range(E):
+            out = _swiglu_loops(x[t], wgu[e, :f], wgu[e, f:], wd[e])
+            w = weight.get(e, 0.0)
+            for i in range(d):
+                y[t, i] += w * out[i]
+    return y
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("k", [1, 2, 5])
+def test_expert_loop_equals_dense_with_zero_weights(mode, k):
+    """[SEV]: the per-expert loop and the dense zero-weight form match.  With
+    k = E = 5 this is also the k = E reduction to sum_e p_e FFN_e(x)."""
+    rng = np.random.default_rng(100 + 10 * mode + k)
+    x, wr, wgu, wd = _layer(rng, T=6, d=5, E=5, f=3)
+    bias = _rand(rng, 5, scale=0.2)
+    y, _, _ = oracle.moe_layer(x, wr, bias, k, mode, _experts(wgu, wd), 5, bias_select_only=1,
+                               decision_dtype=None)
+    ref = _dense_with_zero_weights(x, wr, bias, k, mode, wgu, wd, bias_select_only=1)
+    assert np.max(np.abs(y - ref)) <= 1e-12 * max(1.0, np.max(np.abs(ref)))
+
+
+def test_shared_expert_adds_its_dense_ffn():
+    rng = np.random.default_rng(9)
+    x, wr, wgu, wd = _layer(rng)
+    sg, su, sd = _rand(rng, 4, 6), _rand(rng, 4, 6), _rand(rng, 6, 4)
+    y0, _, _ = oracle.moe_layer(x, wr, None, 2, oracle.SOFTMAX_TOPK, _experts(wgu, wd), 5)
+    y1, _, _ = oracle.moe_layer(x, wr, None, 2, oracle.SOFTMAX_TOPK, _experts(wgu, wd), 5,
+                                shared_weights=[(sg, su, sd)])
+    for t in range(x.shape[0]):
+        assert (y1[t] - y0[t]).tolist() == pytest.approx(_swiglu_loops(x[t], sg, su, sd), rel=1e-12, abs=1e-13)
+
+
+def test_forced_routing_reproduces_free_routing():
+    rng = np.random.default_rng(11)
+    x, wr, wgu, wd = _layer(rng)
+    for mode in MODES:
+        y, r, w = oracle.moe_layer(x, wr, None, 2, mode, _experts(wgu, wd), 5)
+        y2, r2, w2 = oracle.moe_layer(x, wr, None, 2, mode, _experts(wgu, wd), 5, ids=r.ids)
+        assert r2 is None and np.array_equal(y, y2) and np.array_equal(w, w2)
+
+
+def test_token_subsets_are_independent():
+    """Token-choice routing is per token, so any subset of tokens gives the same rows."""
+    rng = np.random.default_rng(12)
+    x, wr, wgu, wd = _layer(rng, T=20)
+    y, _, _ = oracle.moe_layer(x, wr, None, 2, oracle.SOFTMAX_TOPK, _experts(wgu, wd), 5)
+    sub = [3, 7, 19]
+    ys, _, _ = oracle.moe_layer(x[sub], wr, None, 2, oracle.SOFTMAX_TOPK, _experts(wgu, wd), 5)
+    assert np.max(np.abs(ys - y[sub])) <= 1e-12 * np.max(np.abs(y))
+
+
+# ------------------------------------------------------------------ occupancy
+def test_occupancy_closed_form_reproduces_printed_table():
+    g = json.loads((GOLDEN / "occupancy_table.json").read_text())
+    for name, row in g["rows"].items():
+        for b, pct in zip(g["batches"], row["percent"]):
+            got = 100.0 * oracle.occupancy_closed_form(row["k"], row["experts"], b)
+            assert round(got, 1) == pct, (name, b, got)
+    wt = g["weights_read_table"]
+    for b, pct in zip(wt["batches"], wt["percent"]):
+        assert round(100.0 * oracle.occupancy_closed_form(wt["k"], wt["experts"], b), 1) == pct
+
+
+@pytest.mark.parametrize("k,E,B,draws", [(2, 8, 8, 1_000_000), (2, 8, 4, 1_000_000), (8, 256, 16, 40_000)])
+def test_occupancy_monte_carlo_within_page_tolerance(k, E, B, draws):
+    g = json.loads((GOLDEN / "occupancy_table.json").read_text())
+    tol = g["monte_carlo_tolerance_pp"]
+    mc = oracle.occupancy_monte_carlo(k, E, B, draws, seed=B)
+    cf = oracle.occupancy_closed_form(k, E, B)
+    assert abs(100.0 * (mc - cf)) < tol
+
+
+# ------------------------------------------------------------------ parameter accounting
+def test_parameter_counts_reproduce_the_pages():
+    g = json.loads((GOLDEN / "param_counts.json").read_text())
+    toy = g["toy_layer"]
+    args = (toy["d_model"], toy["d_ff"])
+    assert oracle.expert_params(*args, toy["n_matrices"]) == toy["params_per_expert"]
+    assert oracle.moe_layer_params(*args, toy["n_experts"], toy["n_matrices"]) == toy["total_params"]
+    assert oracle.active_params(*args, toy["n_experts"], toy["top_k"], toy["n_matrices"]) == \
+        toy["active_params_per_token"]
+    ge = g["gated_expert"]
+    assert round(oracle.expert_params(ge["d_model"], ge["d_ff"], ge["n_matrices"]) / 1e6, 1) == \
+        ge["params_millions_rounded_1"]
+    rs = g["router_size"]
+    assert oracle.moe_layer_params(rs["d_model"], 0, rs["n_experts"], 3) == rs["router_weights"]
+    ds = g["deepseek_v3_expert"]
+    per = oracle.expert_params(ds["d_model"], ds["d_ff"], ds["n_matrices"])
+    assert round(per / 1e6) == ds["params_per_expert_millions_rounded_0"]
+    assert round(per * ds["layers"] * ds["experts_per_layer"] / 1e9, 1) == ds["all_expert_params_billions_rounded_1"]
+
+
+def test_brute_force_exhaustive_tiny_routing():
+    """Every key ordering of 4 experts (with ties), all k: the selected set is
+    the k largest and ties resolve to the lower index."""
+    vals = [0.0, 1.0, 1.0, 2.0]
+    for keyrow in set(itertools.permutations(vals)):
+        key = np.array([keyrow])
+        for k in range(1, 5):
+            ids = oracle.topk_select(key, k)[0].tolist()
+            ranked = sorted(range(4), key=lambda e: (-keyrow[e], e))
+            assert ids == ranked[:k]
