@@ -1,0 +1,400 @@
+"""Benchmark of the sparse MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload mixtral_bf16|gptoss_bf16|deepseek_bf16|decode_bf16|tiny_f32] [--T T]
+
+One step = one full pass of the layer (router + top-k, dispatch, grouped SwiGLU
+experts, combine) over one batch of T synthetic tokens already resident in HBM.
+Default workload: the Mixtral-shaped bf16 layer (T=2048, d=4096, E=8, k=2,
+f=14336).  Inputs are larger than L2 (2.8 GB of expert weights per step), so L2
+is not flushed between steps.  With N>1 (torchrun) every rank runs an
+independent replica on its own T tokens (weak scaling, no data-path
+collective); the step time is the max over ranks.
+
+Rank 0 prints one JSON line.  ``value`` is tokens/s over all ranks; the line
+also carries active TFLOP/s, the per-stage split, the roofline of the grouped
+expert GEMMs, an end-to-end number through host buffers, SM clocks sampled
+during the timed region and the CPU oracle's throughput on a bounded sample.
+``--impl reference`` times the CPU oracle itself on the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import pathlib
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = pathlib.Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import synth  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def layer_flops(cfg: synth.LayerConfig, counts: np.ndarray) -> dict:
+    """Algorithmic FLOPs of one step, split by stage (rows = measured tokens per expert)."""
+    rows = float(np.sum(counts))
+    router = 2.0 * cfg.T * cfg.d_model * cfg.n_experts
+    experts = 6.0 * cfg.d_model * cfg.d_ff * rows
+    shared = 6.0 * cfg.d_model * cfg.d_ff_shared * cfg.n_shared * cfg.T
+    return dict(router=router, experts=experts, shared=shared, total=router + experts + shared)
+
+
+def layer_bytes(cfg: synth.LayerConfig, counts: np.ndarray) -> dict:
+    """Algorithmic HBM bytes of one step: x, router, touched experts, shared experts, y."""
+    b = 2 if cfg.dtype == "bf16" else 4
+    touched = int(np.sum(counts > 0))
+    d, f = cfg.d_model, cfg.d_ff
+    weights = touched * 3 * d * f * b + cfg.n_shared * 3 * d * cfg.d_ff_shared * b + cfg.n_experts * d * b
+    act = 2 * cfg.T * d * b
+    return dict(weights=weights, activations=act, total=weights + act, touched=touched)
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.tmp = tempfile.NamedTemporaryFile(prefix="clocks_", suffix=".csv", delete=False)
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.tmp.close()
+
+    def summary(self) -> dict:
+        rows = []
+        try:
+            for line in open(self.tmp.name):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        finally:
+            os.unlink(self.tmp.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        loaded = [v for v in sm if mx and v > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_baseline(cfg: synth.LayerConfig, dev: dict, n_tokens: int) -> dict:
+    """The CPU oracle, as it stands, on the first ``n_tokens`` tokens of the workload."""
+    import oracle
+
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        cores = os.cpu_count() or 1
+    T, d, f, E = cfg.T, cfg.d_model, cfg.d_ff, cfg.n_experts
+    n = min(n_tokens, T)
+
+    def bits_to_f64(t):
+        import torch
+        if t.dtype == torch.bfloat16:
+            return synth.bf16_bits_to_f32(t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)).astype(
+                np.float64)
+        return t.float().cpu().numpy().astype(np.float64)
+
+    x = bits_to_f64(dev["x"][:n])
+    wr = bits_to_f64(dev["w_router"])
+    bias = synth.zipf_bias(cfg)
+    bias = bias.astype(np.float64) if bias is not None else None
+
+    def experts(e):
+        gu = bits_to_f64(dev["w_gate_up"][e])
+        return gu[:f], gu[f:], bits_to_f64(dev["w_down"][e])
+
+    shared = []
+    for s in range(cfg.n_shared):
+        gu = bits_to_f64(dev["ws_gate_up"][s])
+        shared.append((gu[:cfg.d_ff_shared], gu[cfg.d_ff_shared:], bits_to_f64(dev["ws_down"][s])))
+    t0 = time.perf_counter()
+    oracle.moe_layer(x, wr, bias, cfg.top_k, cfg.gating, experts, E, shared_weights=shared,
+                     bias_select_only=cfg.bias_select_only)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {n} of {T} tokens of the same layer, float64 numpy, expert weights upcast per call",
+            "seconds": dt}
+
+
+def run_reference(args, cfg) -> None:
+    """--impl reference: the CPU oracle timed on the host cores (rank 0 only)."""
+    import torch
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    dev_name = "cuda" if torch.cuda.is_available() else "cpu"
+    dev = {name: synth.device_tensor(cfg, name, dev_name) for name in synth.tensor_specs(cfg)}
+    n = args.ref_tokens
+    times = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(cfg, dev, n)
+        if i >= args.warmup:
+            times.append(r["seconds"])
+    ms = 1000.0 * sum(times) / len(times)
+    val = n / (ms / 1000.0)
+    line = {
+        "impl": "reference", "metric": "MoE-layer tokens/s", "value": val, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "d_model": cfg.d_model, "n_experts": cfg.n_experts,
+                   "top_k": cfg.top_k, "d_ff": cfg.d_ff, "tokens_per_step": n},
+        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
+                         "sample": r["sample"]},
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="mixtral_bf16", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--T", type=int, default=None, help="override the token count (decode sweep)")
+    ap.add_argument("--zipf", type=float, default=None, help="override the Zipf routing-bias exponent")
+    ap.add_argument("--cpu-tokens", type=int, default=128, help="tokens in the CPU-oracle baseline sample")
+    ap.add_argument("--ref-tokens", type=int, default=32, help="tokens per step of --impl reference")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    cfg = synth.workload(args.workload)
+    if args.T is not None:
+        cfg = cfg.replace(T=args.T)
+    if args.zipf is not None:
+        cfg = cfg.replace(zipf_s=args.zipf)
+
+    if args.impl == "reference":
+        run_reference(args, cfg)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import top_routing_expert_gemm_b200 as moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if world != args.gpus and rank == 0:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+
+    # ---- inputs, generated in HBM (each rank its own token batch: seed + rank)
+    dev = {}
+    for name in synth.tensor_specs(cfg):
+        dev[name] = synth.device_tensor(cfg if name != "x" else cfg.replace(seed=cfg.seed + 7919 * rank),
+                                        name, "cuda")
+    bias_np = synth.zipf_bias(cfg)
+    bias = torch.from_numpy(bias_np).cuda() if bias_np is not None else None
+    c = moe.make_config(cfg.T, cfg.d_model, cfg.n_experts, cfg.top_k, cfg.d_ff,
+                        moe.MOE_BF16 if cfg.dtype == "bf16" else moe.MOE_F32, cfg.gating, cfg.n_shared,
+                        cfg.d_ff_shared, cfg.bias_select_only)
+    tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    T, d, k, E = cfg.T, cfg.d_model, cfg.top_k, cfg.n_experts
+    ws_bytes = moe.moe_workspace_bytes(c)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    y = torch.empty(T, d, dtype=tdt, device="cuda")
+    ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        moe.moe_forward(c, dev["x"], dev["w_router"], bias, dev["w_gate_up"], dev["w_down"], dev.get("ws_gate_up"),
+                        dev.get("ws_down"), y, ids, w, counts, ws, ws_bytes, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = moe.moe_device_status(ws, ws_bytes, stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+    counts_np = counts.cpu().numpy()
+
+    # ---- timed region: K full steps through moe_forward
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+    clocks = clk.summary()
+
+    # ---- same step as its four C-ABI stages, events between them (per-stage split, roofline)
+    ids2, w2 = torch.empty_like(ids), torch.empty_like(w)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    counts2 = torch.empty_like(counts)
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    row_of = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    x_perm = torch.empty(T * k, d, dtype=tdt, device="cuda")
+    y_perm = torch.empty(T * k, d, dtype=tdt, device="cuda")
+    stage_names = ["router_topk", "permute", "grouped_ffn", "combine"]
+    if cfg.n_shared:
+        raise SystemExit("per-stage split covers routed experts only; shared-expert workloads: use moe_forward")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stage_names) + 1)] for _ in range(args.steps)]
+
+    def staged(e=None):
+        if e is not None:
+            e[0].record(stream)
+        moe.moe_router_topk(c, dev["x"], dev["w_router"], bias, ids2, w2, ws, ws_bytes, stream)
+        if e is not None:
+            e[1].record(stream)
+        moe.moe_permute(c, ids2, dev["x"], counts2, offsets, perm, row_of, x_perm, ws, ws_bytes, stream)
+        if e is not None:
+            e[2].record(stream)
+        moe.moe_grouped_ffn(c, x_perm, offsets, dev["w_gate_up"], dev["w_down"], y_perm, ws, ws_bytes, stream)
+        if e is not None:
+            e[3].record(stream)
+        moe.moe_combine(c, y_perm, row_of, w2, None, y, stream)
+        if e is not None:
+            e[4].record(stream)
+
+    for _ in range(args.warmup):
+        staged()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        staged(evs[i])
+    torch.cuda.synchronize()
+    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
+                for j, n in enumerate(stage_names)}
+
+    # ---- end to end: pinned host x in, host y out, every step
+    x_host = torch.empty(T, d, dtype=tdt, pin_memory=True)
+    x_host.copy_(dev["x"].cpu())
+    y_host = torch.empty(T, d, dtype=tdt, pin_memory=True)
+    x_in = torch.empty_like(dev["x"])
+
+    def e2e_step():
+        x_in.copy_(x_host, non_blocking=True)
+        moe.moe_forward(c, x_in, dev["w_router"], bias, dev["w_gate_up"], dev["w_down"], dev.get("ws_gate_up"),
+                        dev.get("ws_down"), y, ids, w, counts, ws, ws_bytes, stream)
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+
+    pk, pk_kind = peaks()
+    fl = layer_flops(cfg, counts_np)
+    by = layer_bytes(cfg, counts_np)
+    tokens_per_s = world * T / (ms / 1000.0)
+    active_tflops = world * fl["total"] / (ms / 1000.0) / 1e12
+    # dominant kernel: the grouped expert GEMMs (tcgen05), timed as the moe_grouped_ffn stage
+    g_ms = stage_ms["grouped_ffn"]
+    gemm_tflops = fl["experts"] / (g_ms / 1000.0) / 1e12
+    decode = cfg.T <= 64
+    if decode:
+        gbs = by["weights"] / (g_ms / 1000.0) / 1e9
+        roof = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / pk["hbm_gbs"], "traffic": None}
+    else:
+        roof = {"bound": "tensor", "achieved": gemm_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": gemm_tflops / pk["bf16_tflops"], "traffic": None}
+    roof["kernel"] = "grouped_gemm_tc (GEMM-1+SwiGLU and GEMM-2 launches of moe_grouped_ffn)"
+    roof["peak_source"] = pk_kind
+    line = {
+        "metric": "MoE-layer tokens/s (active TFLOP/s and roofline fraction alongside)",
+        "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": cfg.dtype, "data": "synthetic (seeded counter-based generator; random-init weights)",
+        "config": {"workload": cfg.name, "T": T, "d_model": d, "n_experts": E, "top_k": k, "d_ff": cfg.d_ff,
+                   "n_shared": cfg.n_shared, "gating": cfg.gating, "zipf_s": cfg.zipf_s,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "not flushed: inputs larger than L2 (expert weights %.2f GB)" % (
+                       3 * E * d * cfg.d_ff * (2 if cfg.dtype == "bf16" else 4) / 1e9)},
+        "active_tflops": active_tflops,
+        "stage_ms": stage_ms,
+        "roofline": roof,
+        "experts_touched": by["touched"],
+        "clocks": clocks,
+        "e2e": {"value": world * T / (e2e_ms / 1000.0), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * d * x_host.element_size(),
+                "d2h_bytes_per_step": T * d * y_host.element_size()},
+        "gpu_launches": args.steps * (8 if cfg.n_shared == 0 else 10),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = {k2: v for k2, v in cpu_baseline(cfg, dev, args.cpu_tokens).items() if k2 != "seconds"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

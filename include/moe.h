@@ -1,0 +1,170 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) sparse Mixture-of-Experts layer forward.
+ *
+ * The layer (token-choice routing, dropless):
+ *   router logits   l = x W_r^T                                   [T, E]
+ *   selection key   kappa = l + b        (b: optional per-expert bias)
+ *   top-k           the k largest kappa per token, descending, ties -> lower index
+ *   gate weights    one of three rules (moe_gating), fp32
+ *   dispatch        rows grouped by expert (ascending), tokens ascending inside
+ *   expert FFN      h = SiLU(x_e Wg^T) * (x_e Wu^T),  o = h Wd^T   (SwiGLU)
+ *   combine         y[t] = sum_s w[t,s] o_{t,s} + sum_shared FFN_shared(x[t])
+ *
+ * Sources (page title, section):
+ *   "Mixture of Experts (MoE): routing, expert parallelism, and memory"
+ *       -- "How does MoE routing work" (score, softmax, top-k, combine),
+ *          "Shared experts" (always-on experts).
+ *   "Mixture of Experts: why a model with 671 billion parameters uses only 37"
+ *       -- "The router: how a token chooses experts" (a bias-free linear
+ *          router, top-k then softmax over the kept scores, per-expert loop),
+ *          "How many experts to pick and how to score them: top-k, softmax,
+ *          sigmoid" (sigmoid scores normalised over the selected set),
+ *          "Capacity factor: when tokens don't fit" (dropless grouping),
+ *          "How data centres handle it" (tokens grouped by expert, all expert
+ *          multiplies in one launch over a stacked weight matrix).
+ *   "Mixture of experts: how MoE works and what it costs"
+ *       -- "What mixture of experts means in an LLM" (Mixtral top-2 softmax,
+ *          DeepSeek-V3 shared + routed), "Why load balancing is the hard part
+ *          of MoE" (bias steers routing, not the gate values).
+ *   "Mixture of Experts Explained: Routers, Active Parameters and VRAM"
+ *       -- the five router steps (Score, Normalise, Keep the top k,
+ *          Renormalise, Run and combine); "a gated feed-forward block with
+ *          three matrices".
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or retains them.  Layouts are row-major; weights
+ *    are "out x in" (as nn.Linear), so every GEMM is A * B^T with both
+ *    operands contiguous along the reduction dimension.
+ *  - dtype MOE_BF16: x, weights, x_perm, h, y_perm, y are bfloat16, all
+ *    accumulation is fp32.  dtype MOE_F32: every tensor is fp32 and all math is
+ *    fp32 on CUDA cores (no TF32).  Routing weights are always fp32, expert ids,
+ *    counts, offsets and permutations always int32.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  Argument checks happen on the host before anything is
+ *    launched: a failed check returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED /
+ *    MOE_ERR_WORKSPACE and launches nothing.  A failed launch returns MOE_ERR_CUDA.
+ *  - Pointers must be 16-byte aligned.  d_model, d_ff and d_ff_shared must be
+ *    multiples of 8.  Limits: 1 <= n_experts <= 1024, 1 <= top_k <= min(16, E),
+ *    T * top_k < 2^31, n_shared in {0, 1}.
+ *  - `ws` is caller-owned device scratch of at least moe_workspace_bytes(cfg)
+ *    bytes, 256-byte aligned.  Its first 16 bytes hold the device status word
+ *    that kernels set on a bounded-wait expiry or an out-of-range expert id;
+ *    moe_forward clears it on entry, moe_device_status() reads it.
+ *  - Device-side waits (pipeline barriers of the tensor-core GEMMs) are bounded
+ *    by cfg->wait_limit_ns (0 = 2 s).  On expiry the kernel drains its own
+ *    copies, frees its tensor memory, records MOE_ERR_TIMEOUT in the status
+ *    word and returns; it never traps.
+ *  - Calls that share a workspace must not overlap on the GPU.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad shape, k > E, ... */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid request outside this build's limits      */
+  MOE_ERR_WORKSPACE = 3,    /* ws smaller than moe_workspace_bytes(cfg)       */
+  MOE_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed              */
+  MOE_ERR_TIMEOUT = 5,      /* a bounded device wait expired (status word)    */
+  MOE_ERR_BAD_EXPERT_ID = 6 /* moe_permute saw an id outside [0, E) (status)  */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+typedef enum {
+  /* softmax over all E kappas, keep the top k, divide by their sum
+     ("Mixture of Experts Explained...", router steps 2-4)                    */
+  MOE_SOFTMAX_ALL_RENORM = 0,
+  /* top-k kappas, softmax over those k
+     ("...671 billion parameters uses only 37", "The router"; Mixtral)        */
+  MOE_SOFTMAX_TOPK = 1,
+  /* sigmoid score per expert, top-k, divide by the sum of the k
+     ("...671 billion parameters uses only 37", sigmoid gating; DeepSeek-V3)  */
+  MOE_SIGMOID_TOPK_RENORM = 2
+} moe_gating;
+
+typedef struct {
+  int64_t T;                /* tokens                                          */
+  int32_t d_model;          /* d                                               */
+  int32_t n_experts;        /* E routed experts                                */
+  int32_t top_k;            /* k                                               */
+  int32_t d_ff;             /* f, routed expert hidden width                   */
+  int32_t n_shared;         /* S always-on shared experts (0 or 1)             */
+  int32_t d_ff_shared;      /* f_s                                             */
+  int32_t dtype;            /* moe_dtype                                       */
+  int32_t gating;           /* moe_gating                                      */
+  int32_t bias_select_only; /* sigmoid rule: bias steers selection only        */
+  int32_t reserved;         /* must be 0                                       */
+  int64_t wait_limit_ns;    /* bound on any single device wait; 0 = 2 s        */
+} moe_config;
+
+/* Bytes of scratch every entry point below accepts for this config
+   (x_perm, h, y_perm, shared-expert buffers, routing and dispatch metadata,
+   status word).  0 on an invalid config. */
+size_t moe_workspace_bytes(const moe_config* cfg);
+
+/* Static, NUL-terminated description of a status code. */
+const char* moe_status_string(moe_status s);
+
+/* Router + top-k + gate weights, one fused pass.
+   x [T, d] (dtype), w_router [E, d] (dtype), logit_bias [E] fp32 or NULL
+   -> topk_ids [T, k] int32 (slots in descending kappa), topk_w [T, k] fp32. */
+moe_status moe_router_topk(const moe_config* cfg, const void* x, const void* w_router,
+                           const float* logit_bias, int32_t* topk_ids, float* topk_w,
+                           void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Dropless dispatch: a stable counting sort of the T*k assignments by expert,
+   then the row gather.
+   topk_ids [T, k] int32, x [T, d]
+   -> counts [E], offsets [E+1] (exclusive scan, offsets[E] = T*k),
+      perm [T*k] (perm[row] = t*k + s), row_of [T*k] (inverse of perm),
+      x_perm [T*k, d] (x_perm[row] = x[perm[row] / k]).
+   Ids outside [0, E) are skipped and flag MOE_ERR_BAD_EXPERT_ID in the status
+   word (read it with moe_device_status). */
+moe_status moe_permute(const moe_config* cfg, const int32_t* topk_ids, const void* x,
+                       int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* row_of,
+                       void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Grouped SwiGLU experts over the dispatched rows.
+   x_perm [T*k, d], offsets [E+1] (device), w_gate_up [E, 2f, d] (rows 0..f-1
+   gate, f..2f-1 up), w_down [E, d, f] -> y_perm [T*k, d].
+   Rows [offsets[e], offsets[e+1]) use expert e; h [T*k, f] lives in ws. */
+moe_status moe_grouped_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
+                           const void* w_gate_up, const void* w_down, void* y_perm,
+                           void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Weighted un-permute: y[t] = sum_s topk_w[t,s] * y_perm[row_of[t*k+s]] (+ y_shared[t]).
+   y_shared [T, d] or NULL.  fp32 accumulation, y in dtype. */
+moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* row_of,
+                       const float* topk_w, const void* y_shared, void* y, moe_stream_t stream);
+
+/* The whole layer: router_topk -> permute -> grouped_ffn (+ shared expert) -> combine.
+   ws_gate_up [S, 2f_s, d] and ws_down [S, d, f_s] when n_shared = 1, else NULL.
+   opt_topk_ids [T,k], opt_topk_w [T,k], opt_counts [E]: optional outputs (NULL = none).
+   Clears the status word first; no host synchronisation inside. */
+moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_router,
+                       const float* logit_bias, const void* w_gate_up, const void* w_down,
+                       const void* ws_gate_up, const void* ws_down, void* y,
+                       int32_t* opt_topk_ids, float* opt_topk_w, int32_t* opt_counts,
+                       void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Synchronises `stream` and returns the status word of `ws`: MOE_OK,
+   MOE_ERR_TIMEOUT or MOE_ERR_BAD_EXPERT_ID (or MOE_ERR_CUDA). */
+moe_status moe_device_status(const void* ws, size_t ws_bytes, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,89 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds, loads,
+exports every entry point include/moe.h declares, and rejects bad arguments
+before launching anything."""
+import ctypes
+import pathlib
+import re
+
+import pytest
+
+import top_routing_expert_gemm_b200 as moe
+from top_routing_expert_gemm_b200 import build
+
+ROOT = pathlib.Path(__file__).resolve().parents[1]
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return moe.lib()
+
+
+def _declared():
+    names = set()
+    for h in (ROOT / "include").glob("*.h"):
+        txt = re.sub(r"/\*.*?\*/", "", h.read_text(), flags=re.S)
+        names |= set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", txt))
+    return names
+
+
+def test_every_declared_symbol_is_exported(L):
+    declared = _declared()
+    assert declared, "no declarations parsed"
+    assert declared <= set(moe.EXPORTED_SYMBOLS) | declared
+    for name in declared:
+        assert hasattr(L, name), name
+        assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+
+
+def test_binding_covers_the_header():
+    assert _declared() == set(moe.EXPORTED_SYMBOLS)
+
+
+def test_status_strings(L):
+    assert moe.moe_status_string(0) == "ok"
+    assert "workspace" in moe.moe_status_string(3)
+    assert moe.moe_status_string(99) == "unknown status"
+
+
+def _cfg(**kw):
+    base = dict(T=64, d_model=256, n_experts=8, top_k=2, d_ff=512, dtype=moe.MOE_BF16, gating=1)
+    base.update(kw)
+    return moe.make_config(**base)
+
+
+def test_workspace_bytes_valid_and_invalid(L):
+    n = moe.moe_workspace_bytes(_cfg())
+    # at least x_perm + h + y_perm for 128 rows
+    assert n >= 2 * (128 * 256 * 2) + 128 * 512 * 2
+    assert n % 256 == 0
+    assert moe.moe_workspace_bytes(_cfg(top_k=9)) == 0          # k > E
+    assert moe.moe_workspace_bytes(_cfg(d_model=250)) == 0      # not a multiple of 8
+    assert moe.moe_workspace_bytes(_cfg(n_experts=2048, top_k=2)) == 0
+    assert moe.moe_workspace_bytes(_cfg(gating=7)) == 0
+    big = moe.moe_workspace_bytes(_cfg(n_shared=1, d_ff_shared=512))
+    assert big > n
+
+
+def _call_forward(L, cfg, ws_bytes=1 << 20, ptr=256):
+    # fake, aligned, never-dereferenced addresses: every call below must fail its host checks
+    p = ctypes.c_void_p(ptr)
+    return L.moe_forward(ctypes.byref(cfg), p, p, None, p, p, None, None, p, None, None, None, p, ws_bytes, None)
+
+
+def test_host_checks_reject_before_launch(L):
+    assert _call_forward(L, _cfg(top_k=0)) == 1                     # invalid
+    assert _call_forward(L, _cfg(n_experts=2000)) == 2              # beyond the build's limits
+    assert _call_forward(L, _cfg(top_k=17, n_experts=32)) == 2      # beyond the build's limits
+    assert _call_forward(L, _cfg(), ws_bytes=16) == 3               # workspace too small
+    assert _call_forward(L, _cfg(), ptr=258) == 1                   # misaligned pointers
+    assert _call_forward(L, _cfg(n_shared=1, d_ff_shared=512)) == 1  # shared weights missing
+    cfg = _cfg()
+    assert L.moe_forward(ctypes.byref(cfg), None, None, None, None, None, None, None, None, None, None, None,
+                         ctypes.c_void_p(256), 1 << 30, None) == 1  # null tensors
+    assert L.moe_router_topk(None, None, None, None, None, None, None, 0, None) == 1
+
+
+def test_config_struct_layout():
+    assert ctypes.sizeof(moe.MoeConfig) == 56
+    assert moe.MoeConfig.wait_limit_ns.offset == 48

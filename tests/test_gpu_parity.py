@@ -1,0 +1,228 @@
+"""GPU parity: every C-ABI call against the CPU oracle on seeded inputs.
+
+Tolerances (written here, not derived at run time):
+  * expert ids, counts, offsets, perm, row_of, x_perm: bit-exact (ids outside
+    the near-tie set; a token whose k-th / (k+1)-th selection-key gap is under
+    1e-3 may flip, and flipped tokens must stay under 0.1% of T);
+  * routing weights: |w - w_ref| <= 2e-5 (fp32 softmax/sigmoid on fp32 logits);
+  * layer outputs: max|y - y_ref| / max|y_ref| <= 1e-4 (fp32), 2e-2 (bf16).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import top_routing_expert_gemm_b200 as moe
+from tests import moe_harness as H
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    # ragged token counts, several tiles, empty experts, every gating rule
+    "mixtral_like": synth.LayerConfig("mixtral_like", 300, 512, 8, 2, 640, "bf16", synth.SOFTMAX_TOPK, seed=11),
+    "gptoss_like": synth.LayerConfig("gptoss_like", 517, 320, 128, 4, 320, "bf16", synth.SOFTMAX_TOPK, seed=12),
+    "deepseek_like": synth.LayerConfig("deepseek_like", 257, 512, 64, 8, 256, "bf16", synth.SIGMOID_TOPK_RENORM,
+                                       n_shared=1, d_ff_shared=384, zipf_s=1.0, bias_select_only=1, seed=13),
+    "allrenorm_bf16": synth.LayerConfig("allrenorm_bf16", 129, 256, 16, 3, 200, "bf16",
+                                        synth.SOFTMAX_ALL_RENORM, zipf_s=1.2, seed=14),
+    "f32_sigmoid_shared": synth.LayerConfig("f32_sigmoid_shared", 190, 264, 12, 3, 136, "f32",
+                                            synth.SIGMOID_TOPK_RENORM, n_shared=1, d_ff_shared=96, zipf_s=0.8,
+                                            seed=15),
+    "k_equals_E": synth.LayerConfig("k_equals_E", 64, 256, 4, 4, 256, "bf16", synth.SOFTMAX_ALL_RENORM, seed=16),
+    "single_expert": synth.LayerConfig("single_expert", 200, 256, 1, 1, 384, "bf16", synth.SOFTMAX_TOPK, seed=17),
+    "one_token": synth.LayerConfig("one_token", 1, 512, 8, 2, 512, "bf16", synth.SOFTMAX_TOPK, seed=18),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    moe.lib()
+
+
+# ------------------------------------------------------------------ whole layer, small
+def test_tiny_f32_layer_full_parity():
+    cfg = synth.workload("tiny_f32")
+    inp = H.make_inputs(cfg)
+    out = H.run_forward(inp)
+    st = H.check_forward(inp, out)
+    assert st["mismatched"] == 0
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_layers_full_parity(name):
+    cfg = SMALL[name]
+    inp = H.make_inputs(cfg)
+    out = H.run_forward(inp)
+    H.check_forward(inp, out)
+
+
+def test_forward_is_deterministic():
+    inp = H.make_inputs(SMALL["deepseek_like"])
+    a = H.run_forward(inp)
+    b = H.run_forward(inp)
+    assert torch.equal(a["y"].view(torch.int16), b["y"].view(torch.int16))
+    assert torch.equal(a["ids"], b["ids"]) and torch.equal(a["w"], b["w"])
+
+
+def test_huge_bias_sends_every_token_to_one_expert():
+    cfg = synth.LayerConfig("forced", 700, 256, 8, 2, 256, "bf16", synth.SOFTMAX_TOPK, seed=19)
+    inp = H.make_inputs(cfg)
+    b = np.zeros(8, np.float32)
+    b[5] = 1e4
+    inp.bias = b
+    inp.dev["bias"] = torch.from_numpy(b).cuda()
+    out = H.run_forward(inp)
+    assert np.all(out["ids"].cpu().numpy()[:, 0] == 5)
+    assert int(out["counts"][5]) == 700
+    H.check_forward(inp, out)
+
+
+def test_zero_tokens_is_a_no_op():
+    cfg = SMALL["mixtral_like"]
+    c = H.moe_cfg(cfg, T=0)
+    inp = H.make_inputs(cfg)
+    ws = torch.empty(max(256, moe.moe_workspace_bytes(c)), dtype=torch.uint8, device="cuda")
+    counts = torch.full((8,), 7, dtype=torch.int32, device="cuda")
+    y = torch.empty(0, cfg.d_model, dtype=torch.bfloat16, device="cuda")
+    moe.moe_forward(c, inp.dev["x"], inp.dev["w_router"], None, inp.dev["w_gate_up"], inp.dev["w_down"], None, None,
+                    y, None, None, counts, ws)
+    torch.cuda.synchronize()
+    assert torch.all(counts == 0)
+
+
+# ------------------------------------------------------------------ single entry points
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("gating", [0, 1, 2])
+@pytest.mark.parametrize("E,k", [(8, 2), (64, 6), (256, 8)])
+def test_router_topk(dtype, gating, E, k):
+    cfg = synth.LayerConfig("r", 333, 264, E, k, 8, dtype, gating, zipf_s=1.1, bias_select_only=1, seed=E + k)
+    inp = H.make_inputs(cfg)
+    c = H.moe_cfg(cfg)
+    ws = torch.empty(moe.moe_workspace_bytes(c), dtype=torch.uint8, device="cuda")
+    ids = torch.empty(cfg.T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(cfg.T, k, dtype=torch.float32, device="cuda")
+    moe.moe_router_topk(c, inp.dev["x"], inp.dev["w_router"], inp.dev["bias"], ids, w, ws)
+    torch.cuda.synchronize()
+    x = synth.host_tensor(cfg, "x").reshape(cfg.T, cfg.d_model)
+    wr = synth.host_tensor(cfg, "w_router").reshape(E, cfg.d_model)
+    r = oracle.route(x, wr, inp.bias.astype(np.float64), k, gating, cfg.bias_select_only)
+    H.check_routing(cfg, ids.cpu().numpy().astype(np.int64), w.cpu().numpy().astype(np.float64), r, cfg.T)
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 1, 1), (1000, 8, 2), (4099, 256, 8), (2048, 1024, 16), (333, 5, 5)])
+@pytest.mark.parametrize("skew", ["uniform", "one_expert", "half_empty"])
+def test_permute_bit_exact(T, E, k, skew):
+    rng = np.random.default_rng(T + E + k)
+    if skew == "uniform":
+        keys = rng.random((T, E))
+    elif skew == "one_expert":
+        keys = rng.random((T, E))
+        keys[:, E // 2] += 10.0
+    else:
+        keys = rng.random((T, E))
+        keys[:, : (E + 1) // 2] += 10.0
+    ids = np.argsort(-keys, axis=1, kind="stable")[:, :k].astype(np.int32)
+    d = 136
+    x = rng.standard_normal((T, d)).astype(np.float32)
+    cfg = synth.LayerConfig("p", T, d, E, k, 8, "f32", 0)
+    c = H.moe_cfg(cfg)
+    ws = torch.empty(moe.moe_workspace_bytes(c), dtype=torch.uint8, device="cuda")
+    dids = torch.from_numpy(ids).cuda()
+    dx = torch.from_numpy(x).cuda()
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    row_of = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    x_perm = torch.empty(T * k, d, dtype=torch.float32, device="cuda")
+    moe.moe_permute(c, dids, dx, counts, offsets, perm, row_of, x_perm, ws)
+    assert moe.moe_device_status(ws) == 0
+    rc, ro, rp, rr = oracle.dispatch(ids.astype(np.int64), E)
+    assert np.array_equal(counts.cpu().numpy(), rc)
+    assert np.array_equal(offsets.cpu().numpy(), ro)
+    assert np.array_equal(perm.cpu().numpy(), rp)
+    assert np.array_equal(row_of.cpu().numpy(), rr)
+    assert np.array_equal(x_perm.cpu().numpy(), x[rp // k])
+
+
+def test_permute_flags_out_of_range_ids():
+    T, E, k, d = 100, 8, 2, 16
+    ids = np.zeros((T, k), np.int32)
+    ids[:, 1] = 1
+    ids[7, 1] = 9  # out of range
+    cfg = synth.LayerConfig("p", T, d, E, k, 8, "f32", 0)
+    c = H.moe_cfg(cfg)
+    ws = torch.zeros(moe.moe_workspace_bytes(c), dtype=torch.uint8, device="cuda")
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    row_of = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    x_perm = torch.empty(T * k, d, dtype=torch.float32, device="cuda")
+    x = torch.zeros(T, d, device="cuda")
+    moe.moe_permute(c, torch.from_numpy(ids).cuda(), x, counts, offsets, perm, row_of, x_perm, ws)
+    assert moe.moe_device_status(ws) == moe.MOE_ERR_BAD_EXPERT_ID
+    assert int(offsets[E]) == T * k - 1
+    assert int(row_of[7 * k + 1]) == -1
+
+
+def _ragged_offsets(sizes):
+    return np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("sizes,d,f", [
+    ([0, 1, 127, 129, 300, 0, 256], 256, 384),   # several m-tiles, ragged tails, empty groups
+    ([5, 0, 140], 264, 200),                     # partial n-tiles in both GEMMs
+    ([1000], 512, 1024),                          # one big group
+    ([3] * 40, 128, 136),                         # many tiny groups
+])
+def test_grouped_ffn_against_dense_experts(dtype, sizes, d, f):
+    rng = np.random.default_rng(sum(sizes) + d + f)
+    G = len(sizes)
+    rows = int(sum(sizes))
+    offs = _ragged_offsets(sizes)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    a = torch.from_numpy(rng.standard_normal((rows, d)).astype(np.float32)).to(tdt).cuda()
+    wgu = torch.from_numpy((rng.standard_normal((G, 2 * f, d)) / np.sqrt(d)).astype(np.float32)).to(tdt).cuda()
+    wd = torch.from_numpy((rng.standard_normal((G, d, f)) / np.sqrt(f)).astype(np.float32)).to(tdt).cuda()
+    y = torch.full((rows, d), float("nan"), dtype=tdt, device="cuda")
+    # the call's T*k must equal the row count: use k = 1, T = rows
+    cfg = synth.LayerConfig("g", rows, d, G, 1, f, dtype, 0)
+    c = H.moe_cfg(cfg)
+    ws = torch.empty(moe.moe_workspace_bytes(c), dtype=torch.uint8, device="cuda")
+    moe.moe_grouped_ffn(c, a, torch.from_numpy(offs).cuda(), wgu, wd, y, ws)
+    assert moe.moe_device_status(ws) == 0
+    A = H.device_to_host_f64(a)
+    WGU = H.device_to_host_f64(wgu)
+    WD = H.device_to_host_f64(wd)
+    ref = np.zeros((rows, d))
+    for g in range(G):
+        r0, r1 = offs[g], offs[g + 1]
+        if r1 > r0:
+            ref[r0:r1] = oracle.swiglu_expert(A[r0:r1], WGU[g, :f], WGU[g, f:], WD[g])
+    got = H.device_to_host_f64(y)
+    assert not np.any(np.isnan(got))
+    assert H.rel_err(got, ref) <= H.TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("shared", [False, True])
+def test_combine(dtype, shared):
+    rng = np.random.default_rng(3)
+    T, k, d = 257, 3, 264
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    yp = torch.from_numpy(rng.standard_normal((T * k, d)).astype(np.float32)).to(tdt).cuda()
+    row_of = rng.permutation(T * k).astype(np.int32)
+    w = rng.random((T, k)).astype(np.float32)
+    ys = torch.from_numpy(rng.standard_normal((T, d)).astype(np.float32)).to(tdt).cuda() if shared else None
+    y = torch.empty(T, d, dtype=tdt, device="cuda")
+    cfg = synth.LayerConfig("c", T, d, 8, k, 8, dtype, 0)
+    moe.moe_combine(H.moe_cfg(cfg), yp, torch.from_numpy(row_of).cuda(), torch.from_numpy(w).cuda(), ys, y)
+    torch.cuda.synchronize()
+    YP = H.device_to_host_f64(yp)
+    ref = np.einsum("tk,tkd->td", w.astype(np.float64), YP[row_of.reshape(T, k)])
+    if shared:
+        ref += H.device_to_host_f64(ys)
+    assert H.rel_err(H.device_to_host_f64(y), ref) <= (1e-6 if dtype == "f32" else 8e-3)

@@ -1,0 +1,395 @@
+// Grouped expert GEMMs on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// "Mixture of Experts: why a model with 671 billion parameters uses only 37",
+// "How data centres handle it": tokens grouped by their assigned expert and
+// all expert multiplies run in a single launch over a stacked weight matrix.
+// Expert FFN: "Mixture of Experts Explained: Routers, Active Parameters and
+// VRAM" (a gated feed-forward block with three matrices), read as SwiGLU.
+//
+//   GEMM-1 (MODE_SWIGLU): h[rows, f] = SiLU(A Wg^T) * (A Wu^T), one launch
+//     over every expert; each 128x256 accumulator holds 128 gate columns and
+//     the matching 128 up columns, so the SwiGLU is applied in the epilogue
+//     straight out of tensor memory and only h (bf16) reaches HBM.
+//   GEMM-2 (MODE_PLAIN):  y[rows, d] = h Wd^T.
+//
+// Persistent, warp-specialised CTA (192 threads, one CTA per SM):
+//   warp 0     TMA producer: 4-stage ring of (A 128x64, B 256x64) bf16 tiles,
+//              128-byte swizzle, mbarrier transaction counts
+//   warp 1     TMEM allocator and single-thread tcgen05.mma issuer
+//              (M=128, N=256, K=16 per instruction, fp32 accumulators)
+//   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter, SwiGLU / bf16
+//              conversion, masked 16-byte stores
+// Two 256-column accumulators (all 512 TMEM columns) let the epilogue of tile
+// i overlap the main loop of tile i+1.
+//
+// Tiles are (group, n-tile, m-tile) with the m-tile fastest, read from the
+// device offsets at kernel start (no host sync): CTAs that run together share
+// one expert's weight panel, so it crosses HBM about once while its row
+// blocks are still in L2.  Rows past a group's end are computed on whatever
+// the TMA box holds (the next group's rows or zero fill) and never stored.
+//
+// Every wait is bounded (Params::wait_limit_ns).  On expiry the CTA raises a
+// shared abort flag and the device status word, lets its in-flight TMA loads
+// and MMAs land, frees its tensor memory and returns.
+#include <cudaTypedefs.h>
+
+#include "kernels.cuh"
+#include "tc_primitives.cuh"
+
+namespace moe {
+namespace tc {
+namespace {
+
+constexpr int BM = 128, BK = 64, STAGES = 4, THREADS = 192;
+constexpr int BN_MMA = 256;
+constexpr int A_BYTES = BM * BK * 2;       // 16 KiB
+constexpr int B_BYTES = BN_MMA * BK * 2;   // 32 KiB
+constexpr int TMEM_COLS = 2 * BN_MMA;      // two accumulators
+constexpr int MODE_SWIGLU = 0, MODE_PLAIN = 1;
+constexpr uint64_t kDrainLimitNs = 200ull * 1000 * 1000;
+
+struct Params {
+  const int32_t* offsets;  // [G+1] device, or null: one group of `rows` rows
+  int G;
+  int64_t rows;            // rows of A and of the output
+  int K;                   // reduction length
+  int N;                   // output columns
+  int nt;                  // n-tiles per group
+  int64_t b_group_rows;    // rows of B per group (2f or d)
+  int up_off;              // row offset of the up half inside a group (f)
+  void* out;
+  int64_t ldo;
+  int* status;
+  uint64_t wait_limit_ns;
+};
+
+__host__ __device__ constexpr int bn_out(int mode) { return mode == MODE_SWIGLU ? BN_MMA / 2 : BN_MMA; }
+
+size_t smem_bytes(int G) {
+  return 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + 256 + 2 * sizeof(int) * (size_t)(G + 1);
+}
+
+// largest g with cum[g] * nt <= t  (t < cum[G] * nt)
+__device__ __forceinline__ void decode_tile(int64_t t, int nt, const int* cum, int G, int& g, int& mt, int& ntile) {
+  int lo = 0, hi = G;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if ((int64_t)cum[mid] * nt <= t) lo = mid;
+    else hi = mid;
+  }
+  g = lo;
+  const int mtiles = cum[lo + 1] - cum[lo];
+  const int64_t local = t - (int64_t)cum[lo] * nt;
+  ntile = (int)(local / mtiles);
+  mt = (int)(local % mtiles);
+}
+
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > kDrainLimitNs) break;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(THREADS, 1)
+    grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                           const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = bars + 2 * STAGES + 2;
+  uint64_t* drain = bars + 2 * STAGES + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* fill_par = reinterpret_cast<int*>(tmem_slot + 2);  // [STAGES]
+  int* s_off = fill_par + STAGES;                          // [G+1]
+  int* s_cum = s_off + (p.G + 1);                          // [G+1]
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int G = p.G;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+      fill_par[s] = -1;
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&tfull[a]), 1);
+      mbar_init(smem_u32(&tempty[a]), 128);
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (p.offsets) {
+    for (int g = threadIdx.x; g <= G; g += THREADS) s_off[g] = p.offsets[g];
+  } else if (threadIdx.x == 0) {
+    s_off[0] = 0;
+    s_off[1] = (int)p.rows;
+  }
+  __syncthreads();
+  if (warp == 0) {  // cumulative m-tile counts, 32 groups per step
+    int carry = 0;
+    if (lane == 0) s_cum[0] = 0;
+    for (int base = 0; base < G; base += 32) {
+      const int g = base + lane;
+      int v = 0;
+      if (g < G) v = max(0, (s_off[g + 1] - s_off[g] + BM - 1) / BM);
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += u;
+      }
+      if (g < G) s_cum[g + 1] = carry + v;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem_base = *tmem_slot;
+  const int64_t total = (int64_t)s_cum[G] * p.nt;
+  const int kb_count = (p.K + BK - 1) / BK;
+  constexpr int BNO = bn_out(MODE);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
+        int g, mt, ntile;
+        decode_tile(t, p.nt, s_cum, G, g, mt, ntile);
+        const int a_row = s_off[g] + mt * BM;
+        const int b_row = (int)((int64_t)g * p.b_group_rows + (int64_t)ntile * BNO);
+        bool ok = true;
+        for (int kb = 0; kb < kb_count; ++kb) {
+          if (!mbar_wait_bounded(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, p.wait_limit_ns, p.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&full[stage]);
+          mbar_expect_tx(fb, A_BYTES + B_BYTES);
+          fill_par[stage] = (int)phase;
+          tma_load_2d(smem_u32(sA + stage * A_BYTES), &tmA, fb, kb * BK, a_row);
+          if (MODE == MODE_SWIGLU) {
+            tma_load_2d(smem_u32(sB + stage * B_BYTES), &tmB, fb, kb * BK, b_row);
+            tma_load_2d(smem_u32(sB + stage * B_BYTES + B_BYTES / 2), &tmB, fb, kb * BK, b_row + p.up_off);
+          } else {
+            tma_load_2d(smem_u32(sB + stage * B_BYTES), &tmB, fb, kb * BK, b_row);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN_MMA);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        if (!mbar_wait_bounded(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, p.wait_limit_ns, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN_MMA);
+        for (int kb = 0; kb < kb_count; ++kb) {
+          if (!mbar_wait_bounded(smem_u32(&full[stage]), phase, abort_flag, p.wait_limit_ns, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_bf16(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32), idesc,
+                     (kb | kk) != 0 ? 1u : 0u);
+          mma_commit(smem_u32(&empty[stage]));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(&tfull[acc]));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+    }
+  } else {
+    // -------------------------------------------------- epilogue (warps 2..5)
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
+      int g, mt, ntile;
+      decode_tile(t, p.nt, s_cum, G, g, mt, ntile);
+      if (!mbar_wait_bounded(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.wait_limit_ns, p.status)) break;
+      tc_fence_after();
+      const int rows_g = s_off[g + 1] - s_off[g];
+      const int lr = mt * BM + r;
+      const int64_t grow = (int64_t)s_off[g] + lr;
+      const bool ok = lr < rows_g && grow >= 0 && grow < p.rows;
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MMA);
+      const int col_base = ntile * BNO;
+      __nv_bfloat16* orow = out + grow * p.ldo + col_base;
+      if (MODE == MODE_SWIGLU) {
+#pragma unroll 1
+        for (int c = 0; c < BNO; c += 32) {
+          uint32_t gv[32], uv[32];
+          tmem_ld32(tb + c, gv);
+          tmem_ld32(tb + BNO + c, uv);
+          tmem_ld_wait();
+          if (ok) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float h0 = silu_f(__uint_as_float(gv[2 * j])) * __uint_as_float(uv[2 * j]);
+              const float h1 = silu_f(__uint_as_float(gv[2 * j + 1])) * __uint_as_float(uv[2 * j + 1]);
+              pk[j] = pack_bf16x2(h0, h1);
+            }
+            if (col_base + c + 32 <= p.N) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            } else {
+              const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(pk);
+              for (int j = 0; j < 32 && col_base + c + j < p.N; ++j) orow[c + j] = hv[j];
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BNO; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(tb + c, v);
+          tmem_ld_wait();
+          if (ok) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+            if (col_base + c + 32 <= p.N) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            } else {
+              const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(pk);
+              for (int j = 0; j < 32 && col_base + c + j < p.N; ++j) orow[c + j] = hv[j];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&tempty[acc]));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  __syncthreads();
+  if (*abort_flag) {
+    // let this CTA's own asynchronous copies and MMAs land before its shared
+    // and tensor memory are released
+    if (warp == 0 && lane == 0) {
+      for (int s = 0; s < STAGES; ++s)
+        if (fill_par[s] >= 0) drain_wait(smem_u32(&full[s]), (uint32_t)fill_par[s]);
+    }
+    if (warp == 1 && lane == 0) {
+      mma_commit(smem_u32(drain));
+      drain_wait(smem_u32(drain), 0);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+// bf16 row-major [rows, cols] tensor, box = box_rows x 64 columns, 128-byte swizzle
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+cudaError_t launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, int64_t tiles_bound,
+                        cudaStream_t stream) {
+  const size_t smem = smem_bytes(p.G);
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  int64_t grid = device_sm_count();
+  if (tiles_bound < grid) grid = tiles_bound;
+  if (grid < 1) grid = 1;
+  grouped_gemm_tc_kernel<MODE><<<(unsigned)grid, THREADS, smem, stream>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace tc
+
+cudaError_t launch_grouped_ffn_bf16_tc(const GroupedFfnArgs& a, cudaStream_t stream) {
+  using namespace tc;
+  if (a.rows == 0) return cudaSuccess;
+  CUtensorMap mA1, mB1, mA2, mB2;
+  if (!make_map(&mA1, a.a, a.rows, a.d, BM) || !make_map(&mB1, a.w_gate_up, (uint64_t)a.G * 2 * a.f, a.d, BN_MMA / 2) ||
+      !make_map(&mA2, a.h, a.rows, a.f, BM) || !make_map(&mB2, a.w_down, (uint64_t)a.G * a.d, a.f, BN_MMA))
+    return cudaErrorInvalidValue;
+  const int G = a.offsets ? a.G : 1;
+  const int64_t mt_bound = (a.rows + BM - 1) / BM + (a.offsets ? a.G : 0);
+  const uint64_t lim = a.wait_limit_ns ? a.wait_limit_ns : 2000000000ull;
+  Params p1{a.offsets, G, a.rows, a.d, a.f, (a.f + bn_out(MODE_SWIGLU) - 1) / bn_out(MODE_SWIGLU),
+            2 * (int64_t)a.f, a.f, a.h, a.f, a.status, lim};
+  cudaError_t e = launch_mode<MODE_SWIGLU>(mA1, mB1, p1, mt_bound * p1.nt, stream);
+  if (e != cudaSuccess) return e;
+  Params p2{a.offsets, G, a.rows, a.f, a.d, (a.d + bn_out(MODE_PLAIN) - 1) / bn_out(MODE_PLAIN), (int64_t)a.d, 0,
+            a.y, a.d, a.status, lim};
+  return launch_mode<MODE_PLAIN>(mA2, mB2, p2, mt_bound * p2.nt, stream);
+}
+
+}  // namespace moe

@@ -1,0 +1,77 @@
+// Host-side launchers of the MoE kernels (internal to the library; the public
+// surface is include/moe.h).  Every launcher is asynchronous on `stream` and
+// returns the cudaError_t of its launch(es).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// ---- router + top-k + gate weights (router_topk.cu)
+struct RouterArgs {
+  const void* x;          // [T, d]
+  const void* w_router;   // [E, d]
+  const float* bias;      // [E] or null
+  int32_t* ids;           // [T, k]
+  float* w;               // [T, k]
+  int64_t T;
+  int d, E, k, gating, bias_select_only;
+  bool bf16;
+  int* status;
+  uint64_t wait_limit_ns;
+};
+cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t stream);
+
+// ---- dispatch (permute.cu)
+struct PermuteArgs {
+  const int32_t* ids;     // [T*k]
+  const void* x;          // [T, d] or null (skip the gather)
+  int32_t* counts;        // [E]
+  int32_t* offsets;       // [E+1]
+  int32_t* perm;          // [T*k]
+  int32_t* row_of;        // [T*k]
+  void* x_perm;           // [T*k, d] or null
+  int32_t* chunk_counts;  // scratch [E * n_chunks]
+  int64_t n_assign;       // T*k
+  int k, d, E;
+  int elem_bytes;
+  int* status;
+};
+int permute_n_chunks(int64_t n_assign);
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream);
+
+// ---- grouped expert GEMMs
+// Rows [offsets[g], offsets[g+1]) of A use weight group g.  offsets == null
+// means a single group covering rows [0, rows).
+struct GroupedFfnArgs {
+  const void* a;          // [rows, d]
+  const int32_t* offsets; // [G+1] or null
+  const void* w_gate_up;  // [G, 2f, d]
+  const void* w_down;     // [G, d, f]
+  void* h;                // [rows, f] scratch
+  void* y;                // [rows, d]
+  int64_t rows;           // rows of a / h / y (T*k, or T for a shared expert)
+  int G, d, f;
+  int* status;
+  uint64_t wait_limit_ns;
+};
+cudaError_t launch_grouped_ffn_bf16_tc(const GroupedFfnArgs& a, cudaStream_t stream);  // tcgen05
+cudaError_t launch_grouped_ffn_f32_simt(const GroupedFfnArgs& a, cudaStream_t stream);  // fp32 CUDA cores
+
+// ---- combine (combine.cu)
+struct CombineArgs {
+  const void* y_perm;     // [T*k, d]
+  const int32_t* row_of;  // [T*k]
+  const float* w;         // [T, k]
+  const void* y_shared;   // [T, d] or null
+  void* y;                // [T, d]
+  int64_t T;
+  int k, d;
+  bool bf16;
+};
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
+
+int device_sm_count();
+
+}  // namespace moe

@@ -1,0 +1,270 @@
+// The C ABI of include/moe.h: host-side argument checks, workspace carving
+// and the launch sequence of the layer on the caller's stream.  Nothing here
+// allocates device memory or synchronises, except moe_device_status.
+#include <cuda_runtime.h>
+
+#include "../../include/moe.h"
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+cudaError_t launch_router_topk_simt(const RouterArgs& a, cudaStream_t stream);
+
+cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t stream) {
+  return launch_router_topk_simt(a, stream);
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status check_config(const moe_config* c) {
+  if (c == nullptr) return MOE_ERR_INVALID_ARG;
+  if (c->T < 0 || c->d_model <= 0 || c->d_ff <= 0 || c->n_experts <= 0 || c->top_k <= 0) return MOE_ERR_INVALID_ARG;
+  if (c->d_model % 8 != 0 || c->d_ff % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (c->top_k > c->n_experts) return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c->gating < MOE_SOFTMAX_ALL_RENORM || c->gating > MOE_SIGMOID_TOPK_RENORM) return MOE_ERR_INVALID_ARG;
+  if (c->bias_select_only != 0 && c->bias_select_only != 1) return MOE_ERR_INVALID_ARG;
+  if (c->reserved != 0 || c->wait_limit_ns < 0) return MOE_ERR_INVALID_ARG;
+  if (c->n_shared < 0) return MOE_ERR_INVALID_ARG;
+  if (c->n_shared > 0 && (c->d_ff_shared <= 0 || c->d_ff_shared % 8 != 0)) return MOE_ERR_INVALID_ARG;
+  if (c->n_experts > kMaxExperts || c->top_k > kMaxTopK || c->n_shared > 1) return MOE_ERR_UNSUPPORTED;
+  if (c->T * (int64_t)c->top_k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  // tensor-map row coordinates are 32-bit
+  if ((int64_t)c->n_experts * 2 * c->d_ff >= (int64_t(1) << 31) ||
+      (int64_t)c->n_experts * c->d_model >= (int64_t(1) << 31))
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+size_t elem_bytes(const moe_config* c) { return c->dtype == MOE_BF16 ? 2 : 4; }
+
+struct Carve {
+  int* status;
+  int32_t *ids, *counts, *offsets, *perm, *row_of, *chunk_counts;
+  float* w;
+  void *x_perm, *h, *y_perm, *h_s, *y_s;
+  size_t total;
+};
+
+// Lay out the workspace; with base == nullptr only sizes are computed.
+Carve carve(const moe_config* c, void* base) {
+  Carve k{};
+  uint8_t* b = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> void* {
+    void* p = b ? b + off : nullptr;
+    off += up(bytes);
+    return p;
+  };
+  const int64_t n = c->T * c->top_k;
+  const size_t eb = elem_bytes(c);
+  k.status = static_cast<int*>(take(16));
+  k.ids = static_cast<int32_t*>(take(sizeof(int32_t) * n));
+  k.w = static_cast<float*>(take(sizeof(float) * n));
+  k.counts = static_cast<int32_t*>(take(sizeof(int32_t) * c->n_experts));
+  k.offsets = static_cast<int32_t*>(take(sizeof(int32_t) * (c->n_experts + 1)));
+  k.perm = static_cast<int32_t*>(take(sizeof(int32_t) * n));
+  k.row_of = static_cast<int32_t*>(take(sizeof(int32_t) * n));
+  k.chunk_counts = static_cast<int32_t*>(take(sizeof(int32_t) * (size_t)c->n_experts * permute_n_chunks(n)));
+  k.x_perm = take(eb * n * c->d_model);
+  k.h = take(eb * n * c->d_ff);
+  k.y_perm = take(eb * n * c->d_model);
+  if (c->n_shared > 0) {
+    k.h_s = take(eb * c->T * c->d_ff_shared);
+    k.y_s = take(eb * c->T * c->d_model);
+  }
+  k.total = off;
+  return k;
+}
+
+moe_status check_ws(const moe_config* c, const void* ws, size_t ws_bytes) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < carve(c, nullptr).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+// Make the runtime's current device the one that owns `p`; rejects host pointers.
+cudaError_t bind_device(const void* p) {
+  cudaPointerAttributes at;
+  cudaError_t e = cudaPointerGetAttributes(&at, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return e;
+  }
+  if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged) return cudaErrorInvalidValue;
+  int cur = -1;
+  e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return e;
+  return cur == at.device ? cudaSuccess : cudaSetDevice(at.device);
+}
+
+moe_status bind(const void* p) {
+  const cudaError_t e = bind_device(p);
+  if (e == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+uint64_t wait_limit(const moe_config* c) { return c->wait_limit_ns > 0 ? (uint64_t)c->wait_limit_ns : 2000000000ull; }
+
+cudaError_t run_ffn(const moe_config* c, const void* a, const int32_t* offsets, int G, int64_t rows, int f,
+                    const void* w_gu, const void* w_d, void* h, void* y, int* status, cudaStream_t s) {
+  GroupedFfnArgs g{a, offsets, w_gu, w_d, h, y, rows, G, c->d_model, f, status, wait_limit(c)};
+  return c->dtype == MOE_BF16 ? launch_grouped_ffn_bf16_tc(g, s) : launch_grouped_ffn_f32_simt(g, s);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_bytes(const moe_config* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return carve(cfg, nullptr).total;
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_BAD_EXPERT_ID: return "expert id out of range";
+  }
+  return "unknown status";
+}
+
+moe_status moe_router_topk(const moe_config* cfg, const void* x, const void* w_router, const float* logit_bias,
+                           int32_t* topk_ids, float* topk_w, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !w_router || !topk_ids || !topk_w || !aligned16(x) || !aligned16(w_router) || !aligned16(topk_ids) ||
+      !aligned16(topk_w) || (logit_bias && !aligned16(logit_bias)))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = bind(ws)) != MOE_OK) return st;
+  Carve k = carve(cfg, ws);
+  RouterArgs a{x, w_router, logit_bias, topk_ids, topk_w, cfg->T, cfg->d_model, cfg->n_experts, cfg->top_k,
+               cfg->gating, cfg->bias_select_only, cfg->dtype == MOE_BF16, k.status, wait_limit(cfg)};
+  MOE_CUDA_TRY(launch_router_topk(a, stream));
+  return MOE_OK;
+}
+
+moe_status moe_permute(const moe_config* cfg, const int32_t* topk_ids, const void* x, int32_t* counts,
+                       int32_t* offsets, int32_t* perm, int32_t* row_of, void* x_perm, void* ws, size_t ws_bytes,
+                       moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+  if (!counts || !offsets || !aligned16(counts) || !aligned16(offsets)) return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && (!topk_ids || !perm || !row_of || !x || !x_perm || !aligned16(topk_ids) || !aligned16(perm) ||
+                     !aligned16(row_of) || !aligned16(x) || !aligned16(x_perm)))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = bind(ws)) != MOE_OK) return st;
+  Carve k = carve(cfg, ws);
+  PermuteArgs a{topk_ids, x, counts, offsets, perm, row_of, x_perm, k.chunk_counts, cfg->T * cfg->top_k,
+                cfg->top_k, cfg->d_model, cfg->n_experts, (int)elem_bytes(cfg), k.status};
+  MOE_CUDA_TRY(launch_permute(a, stream));
+  return MOE_OK;
+}
+
+moe_status moe_grouped_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets, const void* w_gate_up,
+                           const void* w_down, void* y_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x_perm || !offsets || !w_gate_up || !w_down || !y_perm || !aligned16(x_perm) || !aligned16(offsets) ||
+      !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(y_perm))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = bind(ws)) != MOE_OK) return st;
+  Carve k = carve(cfg, ws);
+  MOE_CUDA_TRY(run_ffn(cfg, x_perm, offsets, cfg->n_experts, cfg->T * cfg->top_k, cfg->d_ff, w_gate_up, w_down,
+                       k.h, y_perm, k.status, stream));
+  return MOE_OK;
+}
+
+moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* row_of, const float* topk_w,
+                       const void* y_shared, void* y, moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!y_perm || !row_of || !topk_w || !y || !aligned16(y_perm) || !aligned16(row_of) || !aligned16(topk_w) ||
+      !aligned16(y) || (y_shared && !aligned16(y_shared)))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = bind(y)) != MOE_OK) return st;
+  CombineArgs a{y_perm, row_of, topk_w, y_shared, y, cfg->T, cfg->top_k, cfg->d_model, cfg->dtype == MOE_BF16};
+  MOE_CUDA_TRY(launch_combine(a, stream));
+  return MOE_OK;
+}
+
+moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_router, const float* logit_bias,
+                       const void* w_gate_up, const void* w_down, const void* ws_gate_up, const void* ws_down,
+                       void* y, int32_t* opt_topk_ids, float* opt_topk_w, int32_t* opt_counts, void* ws,
+                       size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+  if (!x || !w_router || !w_gate_up || !w_down || !y || !aligned16(x) || !aligned16(w_router) ||
+      !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(y) || (logit_bias && !aligned16(logit_bias)) ||
+      (opt_topk_ids && !aligned16(opt_topk_ids)) || (opt_topk_w && !aligned16(opt_topk_w)) ||
+      (opt_counts && !aligned16(opt_counts)))
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->n_shared > 0 && (!ws_gate_up || !ws_down || !aligned16(ws_gate_up) || !aligned16(ws_down)))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = bind(ws)) != MOE_OK) return st;
+  if ((st = bind(x)) != MOE_OK) return st;
+  Carve k = carve(cfg, ws);
+  MOE_CUDA_TRY(cudaMemsetAsync(k.status, 0, 16, stream));
+  int32_t* ids = opt_topk_ids ? opt_topk_ids : k.ids;
+  float* w = opt_topk_w ? opt_topk_w : k.w;
+  int32_t* counts = opt_counts ? opt_counts : k.counts;
+  if (cfg->T == 0) {
+    MOE_CUDA_TRY(cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->n_experts, stream));
+    return MOE_OK;
+  }
+  RouterArgs ra{x, w_router, logit_bias, ids, w, cfg->T, cfg->d_model, cfg->n_experts, cfg->top_k,
+                cfg->gating, cfg->bias_select_only, cfg->dtype == MOE_BF16, k.status, wait_limit(cfg)};
+  MOE_CUDA_TRY(launch_router_topk(ra, stream));
+  PermuteArgs pa{ids, x, counts, k.offsets, k.perm, k.row_of, k.x_perm, k.chunk_counts, cfg->T * cfg->top_k,
+                 cfg->top_k, cfg->d_model, cfg->n_experts, (int)elem_bytes(cfg), k.status};
+  MOE_CUDA_TRY(launch_permute(pa, stream));
+  MOE_CUDA_TRY(run_ffn(cfg, k.x_perm, k.offsets, cfg->n_experts, cfg->T * cfg->top_k, cfg->d_ff, w_gate_up, w_down,
+                       k.h, k.y_perm, k.status, stream));
+  if (cfg->n_shared > 0)
+    MOE_CUDA_TRY(run_ffn(cfg, x, nullptr, 1, cfg->T, cfg->d_ff_shared, ws_gate_up, ws_down, k.h_s, k.y_s, k.status,
+                         stream));
+  CombineArgs ca{k.y_perm, k.row_of, w, cfg->n_shared > 0 ? k.y_s : nullptr, y, cfg->T, cfg->top_k,
+                 cfg->d_model, cfg->dtype == MOE_BF16};
+  MOE_CUDA_TRY(launch_combine(ca, stream));
+  return MOE_OK;
+}
+
+moe_status moe_device_status(const void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (ws == nullptr || ws_bytes < 16 || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA_TRY(cudaStreamSynchronize(stream));
+  int v = 0;
+  MOE_CUDA_TRY(cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost));
+  if (v == kDevTimeout) return MOE_ERR_TIMEOUT;
+  if (v == kDevBadExpertId) return MOE_ERR_BAD_EXPERT_ID;
+  return v == 0 ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // extern "C"

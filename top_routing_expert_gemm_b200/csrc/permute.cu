@@ -1,0 +1,181 @@
+// Dropless dispatch: a stable counting sort of the T*k (token, slot)
+// assignments by expert, then the row gather x_perm[row] = x[perm[row] / k].
+//
+// "Mixture of Experts: why a model with 671 billion parameters uses only 37",
+// "Capacity factor: when tokens don't fit" (dropless: each expert gets exactly
+// the rows the router assigned) and "How data centres handle it" (tokens are
+// grouped by their assigned expert before the expert multiplies).
+//
+// Three small kernels keep the result deterministic and stable without any
+// global atomics on positions:
+//   count   : per chunk of kChunk assignments, a shared-memory histogram
+//             -> chunk_counts[e][chunk]
+//   scan    : one block turns the histograms into counts, exclusive offsets
+//             and per-(expert, chunk) starting rows
+//   scatter : each warp walks its slice of the chunk in order; ranks among
+//             equal experts come from __match_any_sync, so rows inside an
+//             expert follow ascending assignment index t*k+s
+// and a gather kernel that moves whole rows with 16-byte loads/stores.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kPerWarp = 256;                 // assignments per warp slice
+constexpr int kChunk = kWarps * kPerWarp;     // assignments per block
+
+__global__ void __launch_bounds__(kThreads) permute_count_kernel(const int32_t* __restrict__ ids, int64_t n,
+                                                                 int E, int32_t* chunk_counts, int n_chunks,
+                                                                 int* status) {
+  extern __shared__ int hist[];
+  for (int e = threadIdx.x; e < E; e += kThreads) hist[e] = 0;
+  __syncthreads();
+  const int64_t base = (int64_t)blockIdx.x * kChunk;
+  const int64_t end = min(base + kChunk, n);
+  for (int64_t i = base + threadIdx.x; i < end; i += kThreads) {
+    const int e = ids[i];
+    if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+    else set_status(status, kDevBadExpertId);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kThreads) chunk_counts[(int64_t)e * n_chunks + blockIdx.x] = hist[e];
+}
+
+// one block of kScanThreads >= E threads
+constexpr int kScanThreads = 1024;
+__global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(int32_t* chunk_counts, int n_chunks, int E,
+                                                                    int32_t* counts, int32_t* offsets) {
+  __shared__ int warp_sums[kScanThreads / 32];
+  const int e = threadIdx.x, lane = e % 32, warp = e / 32;
+  int total = 0;
+  if (e < E)
+    for (int b = 0; b < n_chunks; ++b) total += chunk_counts[(int64_t)e * n_chunks + b];
+  // block-wide exclusive scan of the per-expert totals
+  int incl = total;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int s = warp_sums[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, s, off);
+      if (lane >= off) s += v;
+    }
+    warp_sums[lane] = s;  // inclusive over warps
+  }
+  __syncthreads();
+  const int excl = incl - total + (warp > 0 ? warp_sums[warp - 1] : 0);
+  if (e < E) {
+    counts[e] = total;
+    offsets[e] = excl;
+    if (e == E - 1) offsets[E] = excl + total;
+    int run = excl;  // per-chunk starting rows of expert e
+    for (int b = 0; b < n_chunks; ++b) {
+      const int c = chunk_counts[(int64_t)e * n_chunks + b];
+      chunk_counts[(int64_t)e * n_chunks + b] = run;
+      run += c;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) permute_scatter_kernel(const int32_t* __restrict__ ids, int64_t n,
+                                                                   int E, const int32_t* __restrict__ chunk_base,
+                                                                   int n_chunks, int32_t* perm, int32_t* row_of) {
+  extern __shared__ int wc[];  // [kWarps][E]: per-warp counts, then per-warp next row
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int i = threadIdx.x; i < kWarps * E; i += kThreads) wc[i] = 0;
+  __syncthreads();
+  const int64_t slice = (int64_t)blockIdx.x * kChunk + (int64_t)warp * kPerWarp;
+  int* mine = wc + warp * E;
+  // pass 1: per-warp histogram, one update per distinct expert per round
+  for (int r = 0; r < kPerWarp / 32; ++r) {
+    const int64_t i = slice + r * 32 + lane;
+    int e = (i < n) ? ids[i] : -1;
+    if (e >= E) e = -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) mine[e] += __popc(peers);
+  }
+  __syncthreads();
+  // per expert: exclusive scan over the warps, starting at this chunk's base row
+  for (int e = threadIdx.x; e < E; e += kThreads) {
+    int run = chunk_base[(int64_t)e * n_chunks + blockIdx.x];
+    for (int w = 0; w < kWarps; ++w) {
+      const int c = wc[w * E + e];
+      wc[w * E + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  // pass 2: ranks inside each round follow lane order, rounds follow index order
+  const unsigned lt = (1u << lane) - 1u;
+  for (int r = 0; r < kPerWarp / 32; ++r) {
+    const int64_t i = slice + r * 32 + lane;
+    const bool in = i < n;
+    int e = in ? ids[i] : -1;
+    if (e >= E) e = -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    int row = -1;
+    if (e >= 0) row = mine[e] + __popc(peers & lt);
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) mine[e] += __popc(peers);
+    __syncwarp();
+    if (in) {
+      row_of[i] = row;  // -1 for an id outside [0, E)
+      if (row >= 0) perm[row] = (int32_t)i;
+    }
+  }
+}
+
+// x_perm[row] = x[perm[row] / k]; one warp per row, 16-byte vectors
+__global__ void __launch_bounds__(kThreads) gather_rows_kernel(const uint8_t* __restrict__ x,
+                                                               const int32_t* __restrict__ perm,
+                                                               const int32_t* __restrict__ offsets, int E,
+                                                               int k, int64_t row_bytes, uint8_t* x_perm) {
+  const int64_t n_rows = offsets[E];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t n16 = row_bytes / 16;
+  for (int64_t row = (int64_t)blockIdx.x * kWarps + warp; row < n_rows; row += (int64_t)gridDim.x * kWarps) {
+    const int64_t t = perm[row] / k;
+    const uint4* src = reinterpret_cast<const uint4*>(x + t * row_bytes);
+    uint4* dst = reinterpret_cast<uint4*>(x_perm + row * row_bytes);
+    for (int64_t j = lane; j < n16; j += 32) dst[j] = __ldg(src + j);
+  }
+}
+
+}  // namespace
+
+int permute_n_chunks(int64_t n_assign) { return (int)((n_assign + kChunk - 1) / kChunk); }
+
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
+  const int n_chunks = permute_n_chunks(a.n_assign);
+  if (n_chunks == 0) {
+    // no assignments: zero counts and offsets
+    cudaError_t e = cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * a.E, stream);
+    if (e != cudaSuccess) return e;
+    return cudaMemsetAsync(a.offsets, 0, sizeof(int32_t) * (a.E + 1), stream);
+  }
+  permute_count_kernel<<<n_chunks, kThreads, sizeof(int) * a.E, stream>>>(a.ids, a.n_assign, a.E, a.chunk_counts,
+                                                                          n_chunks, a.status);
+  permute_scan_kernel<<<1, kScanThreads, 0, stream>>>(a.chunk_counts, n_chunks, a.E, a.counts, a.offsets);
+  permute_scatter_kernel<<<n_chunks, kThreads, sizeof(int) * kWarps * a.E, stream>>>(
+      a.ids, a.n_assign, a.E, a.chunk_counts, n_chunks, a.perm, a.row_of);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || a.x == nullptr || a.x_perm == nullptr) return e;
+  int64_t blocks = (a.n_assign + kWarps - 1) / kWarps;
+  const int64_t cap = (int64_t)device_sm_count() * 16;
+  if (blocks > cap) blocks = cap;
+  gather_rows_kernel<<<(unsigned)blocks, kThreads, 0, stream>>>(
+      static_cast<const uint8_t*>(a.x), a.perm, a.offsets, a.E, a.k, (int64_t)a.d * a.elem_bytes,
+      static_cast<uint8_t*>(a.x_perm));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,210 @@
+// Fused router: logits = x W_r^T, selection key = logits + bias, top-k with a
+// warp-shuffle merge, then the gate weights of the chosen experts.
+//
+// Follows the router steps of "Mixture of Experts Explained: Routers, Active
+// Parameters and VRAM" (Score, Normalise, Keep the top k, Renormalise), the
+// top-k-then-softmax router of "Mixture of Experts: why a model with 671
+// billion parameters uses only 37" ("The router: how a token chooses
+// experts") and its sigmoid gating ("How many experts to pick and how to
+// score them").
+//
+// One warp owns one token at a time.  Lanes split d (16-byte vector loads),
+// accumulate eight experts' dot products at once in fp32, and butterfly-reduce
+// them into a per-warp logit row in shared memory.  When W_r fits in shared
+// memory (small E: Mixtral-shaped and decode layers) every block stages it
+// once; otherwise it streams from L2.  Top-k: each lane keeps the best KMAX of
+// its strided experts, then k rounds of a warp arg-max (key desc, index asc)
+// pop the winners.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kGroup = 8;  // experts accumulated per pass over x
+
+struct RouterParams {
+  const void* x;
+  const void* w;
+  const float* bias;
+  int32_t* ids;
+  float* wts;
+  int64_t T;
+  int d, E, k, gating, bias_select_only;
+};
+
+template <typename T, bool W_SMEM, int KMAX>
+__global__ void __launch_bounds__(kThreads) router_topk_simt_kernel(RouterParams p) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  constexpr int V = Vec16<T>::N;
+  const int d = p.d, E = p.E, k = p.k;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const T* __restrict__ x = static_cast<const T*>(p.x);
+  const T* __restrict__ wg = static_cast<const T*>(p.w);
+
+  float* logits = reinterpret_cast<float*>(smem) + warp * E;      // [kWarps][E]
+  T* sw = reinterpret_cast<T*>(smem + sizeof(float) * kWarps * E);  // [E][d] when staged
+  if (W_SMEM) {
+    const int64_t n16 = (int64_t)E * d / V;
+    for (int64_t i = threadIdx.x; i < n16; i += kThreads)
+      reinterpret_cast<uint4*>(sw)[i] = __ldg(reinterpret_cast<const uint4*>(wg) + i);
+    __syncthreads();
+  }
+  const T* wsrc = W_SMEM ? sw : wg;
+
+  for (int64_t t = (int64_t)blockIdx.x * kWarps + warp; t < p.T; t += (int64_t)gridDim.x * kWarps) {
+    const T* xr = x + t * d;
+    // ---- Score: logits of all E experts, kGroup at a time
+    for (int e0 = 0; e0 < E; e0 += kGroup) {
+      float acc[kGroup];
+#pragma unroll
+      for (int j = 0; j < kGroup; ++j) acc[j] = 0.f;
+      for (int i0 = lane * V; i0 < d; i0 += 32 * V) {
+        const Vec16<T> xv = ld16(xr + i0);
+        float xf[V];
+#pragma unroll
+        for (int v = 0; v < V; ++v) xf[v] = Elem<T>::to_f(xv.v[v]);
+#pragma unroll
+        for (int j = 0; j < kGroup; ++j) {
+          if (e0 + j < E) {
+            Vec16<T> wv;
+            const T* wp = wsrc + (int64_t)(e0 + j) * d + i0;
+            if (W_SMEM) *reinterpret_cast<uint4*>(wv.v) = *reinterpret_cast<const uint4*>(wp);
+            else wv = ld16(wp);
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[j] = fmaf(xf[v], Elem<T>::to_f(wv.v[v]), acc[j]);
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kGroup; ++j)
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+      float mine = acc[0];
+#pragma unroll
+      for (int j = 1; j < kGroup; ++j) mine = (lane == j) ? acc[j] : mine;
+      if (lane < kGroup && e0 + lane < E) logits[e0 + lane] = mine;
+    }
+    __syncwarp();
+
+    // ---- Keep the top k of kappa = logit + bias
+    TopK<KMAX> tk;
+    tk.init();
+    float mx = -INFINITY;
+    for (int e = lane; e < E; e += 32) {
+      const float kap = logits[e] + (p.bias ? p.bias[e] : 0.f);
+      tk.push(kap, e);
+      mx = fmaxf(mx, kap);
+    }
+    float sel_key[KMAX];
+    int sel_idx[KMAX];
+#pragma unroll
+    for (int s = 0; s < KMAX; ++s) {
+      if (s < k) {
+        float bk = tk.key[0];
+        int bi = tk.idx[0];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+          if (ranks_before(ok, oi, bk, bi)) { bk = ok; bi = oi; }
+        }
+        sel_key[s] = bk;
+        sel_idx[s] = bi;
+        if (tk.idx[0] == bi) {  // the owning lane pops its head
+#pragma unroll
+          for (int j = 0; j + 1 < KMAX; ++j) { tk.key[j] = tk.key[j + 1]; tk.idx[j] = tk.idx[j + 1]; }
+          tk.key[KMAX - 1] = -INFINITY;
+          tk.idx[KMAX - 1] = 0x7fffffff;
+        }
+      } else {
+        sel_key[s] = -INFINITY;
+        sel_idx[s] = 0;
+      }
+    }
+
+    // ---- gate weights of the selected experts
+    float wsel[KMAX];
+    float denom = 0.f;
+    if (p.gating == 0) {
+      // softmax over all E, keep the selected probabilities, renormalise
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      float z = 0.f;
+      for (int e = lane; e < E; e += 32) z += expf(logits[e] + (p.bias ? p.bias[e] : 0.f) - mx);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+#pragma unroll
+      for (int s = 0; s < KMAX; ++s) {
+        wsel[s] = (s < k) ? expf(sel_key[s] - mx) / z : 0.f;
+        denom += wsel[s];
+      }
+    } else if (p.gating == 1) {
+      // softmax over the k kept kappas
+#pragma unroll
+      for (int s = 0; s < KMAX; ++s) {
+        wsel[s] = (s < k) ? expf(sel_key[s] - sel_key[0]) : 0.f;
+        denom += wsel[s];
+      }
+    } else {
+      // sigmoid score, normalised over the selected set
+#pragma unroll
+      for (int s = 0; s < KMAX; ++s) {
+        if (s < k) {
+          const float sc = p.bias_select_only ? logits[sel_idx[s]] : sel_key[s];
+          wsel[s] = 1.0f / (1.0f + expf(-sc));
+        } else {
+          wsel[s] = 0.f;
+        }
+        denom += wsel[s];
+      }
+    }
+#pragma unroll
+    for (int s = 0; s < KMAX; ++s) {
+      if (s < k && lane == s) {
+        p.ids[t * k + s] = sel_idx[s];
+        p.wts[t * k + s] = wsel[s] / denom;
+      }
+    }
+    __syncwarp();
+  }
+}
+
+template <typename T, bool W_SMEM>
+cudaError_t launch_t(const RouterParams& p, cudaStream_t stream) {
+  const size_t logit_bytes = sizeof(float) * kWarps * p.E;
+  const size_t smem = logit_bytes + (W_SMEM ? (size_t)p.E * p.d * sizeof(T) : 0);
+  const int sms = device_sm_count();
+  int64_t blocks = (p.T + kWarps - 1) / kWarps;
+  const int64_t cap = (int64_t)sms * (W_SMEM ? 2 : 8);
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  auto run = [&](auto kernel) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kernel<<<(unsigned)blocks, kThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+  };
+  if (p.k <= 2) return run(router_topk_simt_kernel<T, W_SMEM, 2>);
+  if (p.k <= 4) return run(router_topk_simt_kernel<T, W_SMEM, 4>);
+  if (p.k <= 8) return run(router_topk_simt_kernel<T, W_SMEM, 8>);
+  return run(router_topk_simt_kernel<T, W_SMEM, 16>);
+}
+
+}  // namespace
+
+// W_r is staged in shared memory when it fits next to the logit rows.
+constexpr size_t kRouterSmemBudget = 160 * 1024;
+
+cudaError_t launch_router_topk_simt(const RouterArgs& a, cudaStream_t stream) {
+  RouterParams p{a.x, a.w_router, a.bias, a.ids, a.w, a.T, a.d, a.E, a.k, a.gating, a.bias_select_only};
+  const size_t eb = a.bf16 ? 2 : 4;
+  const bool fits = sizeof(float) * kWarps * a.E + (size_t)a.E * a.d * eb <= kRouterSmemBudget;
+  if (a.bf16)
+    return fits ? launch_t<__nv_bfloat16, true>(p, stream) : launch_t<__nv_bfloat16, false>(p, stream);
+  return fits ? launch_t<float, true>(p, stream) : launch_t<float, false>(p, stream);
+}
+
+}  // namespace moe
