@@ -36,6 +36,7 @@ sys.path.insert(0, str(ROOT))
 
 import synth  # noqa: E402
 
+METRIC = "MoE-layer tokens/s (active TFLOP/s and roofline fraction alongside)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -117,45 +118,88 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def cpu_baseline(cfg: synth.LayerConfig, dev: dict, n_tokens: int) -> dict:
-    """The CPU oracle, as it stands, on the first ``n_tokens`` tokens of the workload."""
-    import oracle
+def config_dict(cfg: synth.LayerConfig, world: int) -> dict:
+    return {"workload": cfg.name, "T": cfg.T, "d_model": cfg.d_model, "n_experts": cfg.n_experts,
+            "top_k": cfg.top_k, "d_ff": cfg.d_ff, "n_shared": cfg.n_shared, "d_ff_shared": cfg.d_ff_shared,
+            "gating": cfg.gating, "zipf_s": cfg.zipf_s,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "not flushed: inputs larger than L2 (expert weights %.2f GB)" % (
+                3 * cfg.n_experts * cfg.d_model * cfg.d_ff * (2 if cfg.dtype == "bf16" else 4) / 1e9)}
 
+
+def _bits_to_f64(t) -> np.ndarray:
+    """Exact float64 copy of a device tensor (bf16 moved as raw bits)."""
+    import torch
+
+    if t.dtype == torch.bfloat16:
+        return synth.bf16_bits_to_f32(t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)).astype(
+            np.float64)
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+class OracleInputs:
+    """The workload's stored inputs as float64 host arrays, the form the oracle reads.
+
+    Expert weights are upcast once up front when they fit in ``prefetch_gb``
+    of host memory (the oracle then runs on resident inputs, like the GPU);
+    otherwise each oracle call upcasts the experts it touches and that time is
+    part of the measurement."""
+
+    def __init__(self, cfg: synth.LayerConfig, dev: dict, n_tokens: int, prefetch_gb: float = 16.0):
+        self.cfg = cfg
+        self.dev = dev
+        self.n = min(n_tokens, cfg.T)
+        self.x = _bits_to_f64(dev["x"][: self.n])
+        self.wr = _bits_to_f64(dev["w_router"])
+        b = synth.zipf_bias(cfg)
+        self.bias = b.astype(np.float64) if b is not None else None
+        fs = cfg.d_ff_shared
+        self.shared = []
+        for s in range(cfg.n_shared):
+            gu = _bits_to_f64(dev["ws_gate_up"][s])
+            self.shared.append((gu[:fs], gu[fs:], _bits_to_f64(dev["ws_down"][s])))
+        per_expert_gb = 3 * cfg.d_model * cfg.d_ff * 8 / 1e9
+        self.prefetched = per_expert_gb * cfg.n_experts <= prefetch_gb
+        self.cache = {e: self._fetch(e) for e in range(cfg.n_experts)} if self.prefetched else None
+
+    def _fetch(self, e: int):
+        f = self.cfg.d_ff
+        gu = _bits_to_f64(self.dev["w_gate_up"][e])
+        return gu[:f], gu[f:], _bits_to_f64(self.dev["w_down"][e])
+
+    def expert(self, e: int):
+        return self.cache[e] if self.cache is not None else self._fetch(e)
+
+    def describe(self) -> str:
+        return (f"first {self.n} of {self.cfg.T} tokens of the same layer, float64 numpy; expert weights "
+                + ("upcast to float64 before timing" if self.prefetched else "upcast inside each timed call"))
+
+
+def cpu_cores() -> int:
     try:
         from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:  # pragma: no cover
-        cores = os.cpu_count() or 1
-    T, d, f, E = cfg.T, cfg.d_model, cfg.d_ff, cfg.n_experts
-    n = min(n_tokens, T)
+        return os.cpu_count() or 1
 
-    def bits_to_f64(t):
-        import torch
-        if t.dtype == torch.bfloat16:
-            return synth.bf16_bits_to_f32(t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)).astype(
-                np.float64)
-        return t.float().cpu().numpy().astype(np.float64)
 
-    x = bits_to_f64(dev["x"][:n])
-    wr = bits_to_f64(dev["w_router"])
-    bias = synth.zipf_bias(cfg)
-    bias = bias.astype(np.float64) if bias is not None else None
+def time_oracle(oi: OracleInputs) -> float:
+    """Seconds for one call of the CPU oracle on the prepared sample."""
+    import oracle
 
-    def experts(e):
-        gu = bits_to_f64(dev["w_gate_up"][e])
-        return gu[:f], gu[f:], bits_to_f64(dev["w_down"][e])
-
-    shared = []
-    for s in range(cfg.n_shared):
-        gu = bits_to_f64(dev["ws_gate_up"][s])
-        shared.append((gu[:cfg.d_ff_shared], gu[cfg.d_ff_shared:], bits_to_f64(dev["ws_down"][s])))
+    cfg = oi.cfg
     t0 = time.perf_counter()
-    oracle.moe_layer(x, wr, bias, cfg.top_k, cfg.gating, experts, E, shared_weights=shared,
-                     bias_select_only=cfg.bias_select_only)
-    dt = time.perf_counter() - t0
-    return {"value": n / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"first {n} of {T} tokens of the same layer, float64 numpy, expert weights upcast per call",
-            "seconds": dt}
+    oracle.moe_layer(oi.x, oi.wr, oi.bias, cfg.top_k, cfg.gating, oi.expert, cfg.n_experts,
+                     shared_weights=oi.shared, bias_select_only=cfg.bias_select_only)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(cfg: synth.LayerConfig, dev: dict, n_tokens: int) -> dict:
+    """The CPU oracle, as it stands, on a bounded sample of the workload."""
+    oi = OracleInputs(cfg, dev, n_tokens)
+    dt = time_oracle(oi)
+    return {"value": oi.n / dt, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": oi.describe(), "seconds": dt}
 
 
 def run_reference(args, cfg) -> None:
@@ -167,20 +211,21 @@ def run_reference(args, cfg) -> None:
         return
     dev_name = "cuda" if torch.cuda.is_available() else "cpu"
     dev = {name: synth.device_tensor(cfg, name, dev_name) for name in synth.tensor_specs(cfg)}
-    n = args.ref_tokens
+    oi = OracleInputs(cfg, dev, args.ref_tokens)
     times = []
     for i in range(args.warmup + args.steps):
-        r = cpu_baseline(cfg, dev, n)
+        dt = time_oracle(oi)
         if i >= args.warmup:
-            times.append(r["seconds"])
+            times.append(dt)
+    n = oi.n
     ms = 1000.0 * sum(times) / len(times)
     val = n / (ms / 1000.0)
+    r = {"cores": cpu_cores(), "sample": oi.describe()}
     line = {
-        "impl": "reference", "metric": "MoE-layer tokens/s", "value": val, "unit": "tokens/s",
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "T": cfg.T, "d_model": cfg.d_model, "n_experts": cfg.n_experts,
-                   "top_k": cfg.top_k, "d_ff": cfg.d_ff, "tokens_per_step": n},
+        "config": dict(config_dict(cfg, args.gpus), oracle_tokens_per_step=n),
         "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
                          "sample": r["sample"]},
         "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -197,6 +242,9 @@ def main() -> None:
     ap.add_argument("--workload", default="mixtral_bf16", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--T", type=int, default=None, help="override the token count (decode sweep)")
     ap.add_argument("--zipf", type=float, default=None, help="override the Zipf routing-bias exponent")
+    ap.add_argument("--set", action="append", default=[], metavar="FIELD=INT",
+                    help="override a shape field of the workload (d_model, d_ff, n_experts, top_k), e.g. for a "
+                         "small profiling case")
     ap.add_argument("--cpu-tokens", type=int, default=128, help="tokens in the CPU-oracle baseline sample")
     ap.add_argument("--ref-tokens", type=int, default=32, help="tokens per step of --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -209,6 +257,14 @@ def main() -> None:
         cfg = cfg.replace(T=args.T)
     if args.zipf is not None:
         cfg = cfg.replace(zipf_s=args.zipf)
+    for kv in args.set:
+        field, val = kv.split("=", 1)
+        if field not in ("d_model", "d_ff", "n_experts", "top_k", "d_ff_shared"):
+            ap.error(f"--set: unknown field {field}")
+        cfg = cfg.replace(**{field: int(val)})
+    if args.set or args.T is not None or args.zipf is not None:
+        cfg = cfg.replace(name=f"{cfg.name}[T={cfg.T},d={cfg.d_model},f={cfg.d_ff},E={cfg.n_experts},"
+                               f"k={cfg.top_k},zipf={cfg.zipf_s}]")
 
     if args.impl == "reference":
         run_reference(args, cfg)
@@ -294,26 +350,38 @@ def main() -> None:
     row_of = torch.empty(T * k, dtype=torch.int32, device="cuda")
     x_perm = torch.empty(T * k, d, dtype=tdt, device="cuda")
     y_perm = torch.empty(T * k, d, dtype=tdt, device="cuda")
-    stage_names = ["router_topk", "permute", "grouped_ffn", "combine"]
+    stage_names = ["router_topk", "permute", "grouped_ffn"] + (["shared_ffn"] if cfg.n_shared else []) + ["combine"]
     if cfg.n_shared:
-        raise SystemExit("per-stage split covers routed experts only; shared-expert workloads: use moe_forward")
+        # the always-on expert as one group over all T tokens
+        c_s = moe.make_config(T, d, 1, 1, cfg.d_ff_shared, c.dtype, cfg.gating)
+        ws_s_bytes = moe.moe_workspace_bytes(c_s)
+        ws_s = torch.zeros(ws_s_bytes, dtype=torch.uint8, device="cuda")
+        off_s = torch.tensor([0, T], dtype=torch.int32, device="cuda")
+        y_sh = torch.empty(T, d, dtype=tdt, device="cuda")
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stage_names) + 1)] for _ in range(args.steps)]
 
     def staged(e=None):
-        if e is not None:
-            e[0].record(stream)
+        j = 0
+
+        def mark():
+            nonlocal j
+            if e is not None:
+                e[j].record(stream)
+            j += 1
+
+        mark()
         moe.moe_router_topk(c, dev["x"], dev["w_router"], bias, ids2, w2, ws, ws_bytes, stream)
-        if e is not None:
-            e[1].record(stream)
+        mark()
         moe.moe_permute(c, ids2, dev["x"], counts2, offsets, perm, row_of, x_perm, ws, ws_bytes, stream)
-        if e is not None:
-            e[2].record(stream)
+        mark()
         moe.moe_grouped_ffn(c, x_perm, offsets, dev["w_gate_up"], dev["w_down"], y_perm, ws, ws_bytes, stream)
-        if e is not None:
-            e[3].record(stream)
-        moe.moe_combine(c, y_perm, row_of, w2, None, y, stream)
-        if e is not None:
-            e[4].record(stream)
+        mark()
+        if cfg.n_shared:
+            moe.moe_grouped_ffn(c_s, dev["x"], off_s, dev["ws_gate_up"], dev["ws_down"], y_sh, ws_s, ws_s_bytes,
+                                stream)
+            mark()
+        moe.moe_combine(c, y_perm, row_of, w2, y_sh if cfg.n_shared else None, y, stream)
+        mark()
 
     for _ in range(args.warmup):
         staged()
@@ -355,8 +423,8 @@ def main() -> None:
     tokens_per_s = world * T / (ms / 1000.0)
     active_tflops = world * fl["total"] / (ms / 1000.0) / 1e12
     # dominant kernel: the grouped expert GEMMs (tcgen05), timed as the moe_grouped_ffn stage
-    g_ms = stage_ms["grouped_ffn"]
-    gemm_tflops = fl["experts"] / (g_ms / 1000.0) / 1e12
+    g_ms = stage_ms["grouped_ffn"] + stage_ms.get("shared_ffn", 0.0)
+    gemm_tflops = (fl["experts"] + fl["shared"]) / (g_ms / 1000.0) / 1e12
     decode = cfg.T <= 64
     if decode:
         gbs = by["weights"] / (g_ms / 1000.0) / 1e9
@@ -365,18 +433,15 @@ def main() -> None:
     else:
         roof = {"bound": "tensor", "achieved": gemm_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": gemm_tflops / pk["bf16_tflops"], "traffic": None}
-    roof["kernel"] = "grouped_gemm_tc (GEMM-1+SwiGLU and GEMM-2 launches of moe_grouped_ffn)"
+    roof["kernel"] = ("grouped_gemm_tc: the GEMM-1+SwiGLU and GEMM-2 launches of moe_grouped_ffn"
+                      + (" (routed and shared experts)" if cfg.n_shared else ""))
     roof["peak_source"] = pk_kind
     line = {
-        "metric": "MoE-layer tokens/s (active TFLOP/s and roofline fraction alongside)",
+        "metric": METRIC,
         "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": cfg.dtype, "data": "synthetic (seeded counter-based generator; random-init weights)",
-        "config": {"workload": cfg.name, "T": T, "d_model": d, "n_experts": E, "top_k": k, "d_ff": cfg.d_ff,
-                   "n_shared": cfg.n_shared, "gating": cfg.gating, "zipf_s": cfg.zipf_s,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "not flushed: inputs larger than L2 (expert weights %.2f GB)" % (
-                       3 * E * d * cfg.d_ff * (2 if cfg.dtype == "bf16" else 4) / 1e9)},
+        "config": config_dict(cfg, world),
         "active_tflops": active_tflops,
         "stage_ms": stage_ms,
         "roofline": roof,

@@ -51,7 +51,9 @@
  *  - `ws` is caller-owned device scratch of at least moe_workspace_bytes(cfg)
  *    bytes, 256-byte aligned.  Its first 16 bytes hold the device status word
  *    that kernels set on a bounded-wait expiry or an out-of-range expert id;
- *    moe_forward clears it on entry, moe_device_status() reads it.
+ *    moe_forward clears it on entry; a caller chaining the single-stage entry
+ *    points zeroes those 16 bytes before the first of them.  moe_device_status()
+ *    reads it.
  *  - Device-side waits (pipeline barriers of the tensor-core GEMMs) are bounded
  *    by cfg->wait_limit_ns (0 = 2 s).  On expiry the kernel drains its own
  *    copies, frees its tensor memory, records MOE_ERR_TIMEOUT in the status

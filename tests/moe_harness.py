@@ -92,17 +92,20 @@ class OracleWeights:
         self._cache = {}
 
     def routed(self, e: int):
-        if e not in self._cache:
-            f = self.cfg.d_ff
-            if self.inp.on_host:
-                d = self.cfg.d_model
-                gu = synth.host_tensor(self.cfg, "w_gate_up", e * 2 * f * d, 2 * f * d).reshape(2 * f, d)
-                wd = synth.host_tensor(self.cfg, "w_down", e * d * f, d * f).reshape(d, f)
-            else:
-                gu = device_to_host_f64(self.inp.dev["w_gate_up"][e])
-                wd = device_to_host_f64(self.inp.dev["w_down"][e])
-            self._cache[e] = (gu[:f], gu[f:], wd)
-        return self._cache[e]
+        if e in self._cache:
+            return self._cache[e]
+        f = self.cfg.d_ff
+        if self.inp.on_host:
+            d = self.cfg.d_model
+            gu = synth.host_tensor(self.cfg, "w_gate_up", e * 2 * f * d, 2 * f * d).reshape(2 * f, d)
+            wd = synth.host_tensor(self.cfg, "w_down", e * d * f, d * f).reshape(d, f)
+        else:
+            gu = device_to_host_f64(self.inp.dev["w_gate_up"][e])
+            wd = device_to_host_f64(self.inp.dev["w_down"][e])
+        w = (gu[:f], gu[f:], wd)
+        if self.inp.on_host:  # full-size experts are refetched rather than held in host memory
+            self._cache[e] = w
+        return w
 
     def shared(self):
         out = []

@@ -1,0 +1,29 @@
+"""Bounded device waits: a wait limit that is certain to expire makes the
+tensor-core GEMMs give up, drain their own copies, free their tensor memory
+and report MOE_ERR_TIMEOUT through the status word -- no trap, no hang -- and
+the next call on the same context runs normally."""
+import pytest
+import torch
+
+import synth
+import top_routing_expert_gemm_b200 as moe
+from tests import moe_harness as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def test_expired_wait_limit_reports_timeout_and_context_survives():
+    # long reductions (d = f = 4096) so that the pipeline's waits outlast a 1 ns limit
+    cfg = synth.LayerConfig("timeout", 1024, 4096, 8, 2, 4096, "bf16", synth.SOFTMAX_TOPK, seed=21)
+    inp = H.make_inputs(cfg)
+    out = H.run_forward(inp, wait_limit_ns=1)
+    assert out["status"] == moe.MOE_ERR_TIMEOUT
+    good = H.run_forward(inp)
+    assert good["status"] == 0
+    H.check_forward(inp, good)

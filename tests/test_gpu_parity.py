@@ -101,7 +101,7 @@ def test_router_topk(dtype, gating, E, k):
     cfg = synth.LayerConfig("r", 333, 264, E, k, 8, dtype, gating, zipf_s=1.1, bias_select_only=1, seed=E + k)
     inp = H.make_inputs(cfg)
     c = H.moe_cfg(cfg)
-    ws = torch.empty(moe.moe_workspace_bytes(c), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(moe.moe_workspace_bytes(c), dtype=torch.uint8, device="cuda")
     ids = torch.empty(cfg.T, k, dtype=torch.int32, device="cuda")
     w = torch.empty(cfg.T, k, dtype=torch.float32, device="cuda")
     moe.moe_router_topk(c, inp.dev["x"], inp.dev["w_router"], inp.dev["bias"], ids, w, ws)
@@ -129,7 +129,7 @@ def test_permute_bit_exact(T, E, k, skew):
     x = rng.standard_normal((T, d)).astype(np.float32)
     cfg = synth.LayerConfig("p", T, d, E, k, 8, "f32", 0)
     c = H.moe_cfg(cfg)
-    ws = torch.empty(moe.moe_workspace_bytes(c), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(moe.moe_workspace_bytes(c), dtype=torch.uint8, device="cuda")
     dids = torch.from_numpy(ids).cuda()
     dx = torch.from_numpy(x).cuda()
     counts = torch.empty(E, dtype=torch.int32, device="cuda")
@@ -191,7 +191,7 @@ def test_grouped_ffn_against_dense_experts(dtype, sizes, d, f):
     # the call's T*k must equal the row count: use k = 1, T = rows
     cfg = synth.LayerConfig("g", rows, d, G, 1, f, dtype, 0)
     c = H.moe_cfg(cfg)
-    ws = torch.empty(moe.moe_workspace_bytes(c), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(moe.moe_workspace_bytes(c), dtype=torch.uint8, device="cuda")
     moe.moe_grouped_ffn(c, a, torch.from_numpy(offs).cuda(), wgu, wd, y, ws)
     assert moe.moe_device_status(ws) == 0
     A = H.device_to_host_f64(a)

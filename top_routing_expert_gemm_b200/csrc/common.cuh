@@ -69,20 +69,23 @@ template <int KMAX>
 struct TopK {
   float key[KMAX];
   int idx[KMAX];
+  float val[KMAX];  // payload carried with each key (the raw logit)
   __device__ __forceinline__ void init() {
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) { key[j] = -INFINITY; idx[j] = 0x7fffffff; }
+    for (int j = 0; j < KMAX; ++j) { key[j] = -INFINITY; idx[j] = 0x7fffffff; val[j] = 0.f; }
   }
-  __device__ __forceinline__ void push(float k, int i) {
+  __device__ __forceinline__ void push(float k, int i, float v = 0.f) {
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
       const bool sw = k > key[j] || (k == key[j] && i < idx[j]);
-      const float tk = key[j];
+      const float tk = key[j], tv = val[j];
       const int ti = idx[j];
       key[j] = sw ? k : tk;
       idx[j] = sw ? i : ti;
+      val[j] = sw ? v : tv;
       k = sw ? tk : k;
       i = sw ? ti : i;
+      v = sw ? tv : v;
     }
   }
 };

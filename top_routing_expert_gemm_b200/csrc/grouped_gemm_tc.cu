@@ -45,7 +45,7 @@ constexpr int BN_MMA = 256;
 constexpr int A_BYTES = BM * BK * 2;       // 16 KiB
 constexpr int B_BYTES = BN_MMA * BK * 2;   // 32 KiB
 constexpr int TMEM_COLS = 2 * BN_MMA;      // two accumulators
-constexpr int MODE_SWIGLU = 0, MODE_PLAIN = 1;
+constexpr int MODE_SWIGLU = 0, MODE_PLAIN = 1, MODE_ROUTER = 2;
 constexpr uint64_t kDrainLimitNs = 200ull * 1000 * 1000;
 
 struct Params {
@@ -61,12 +61,19 @@ struct Params {
   int64_t ldo;
   int* status;
   uint64_t wait_limit_ns;
+  int n_mma;               // MMA N (256, or the padded expert count of the router)
+  // router epilogue only
+  const float* bias;       // [E] or null
+  int32_t* ids;            // [rows, k]
+  float* wts;              // [rows, k]
+  int E, k, gating, bias_select_only;
 };
 
 __host__ __device__ constexpr int bn_out(int mode) { return mode == MODE_SWIGLU ? BN_MMA / 2 : BN_MMA; }
 
-size_t smem_bytes(int G) {
-  return 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + 256 + 2 * sizeof(int) * (size_t)(G + 1);
+size_t smem_bytes(int G, int E) {
+  return 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + 256 + 2 * sizeof(int) * (size_t)(G + 1) +
+         sizeof(float) * (size_t)E;
 }
 
 // largest g with cum[g] * nt <= t  (t < cum[G] * nt)
@@ -90,7 +97,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
     if (globaltimer_ns() - t0 > kDrainLimitNs) break;
 }
 
-template <int MODE>
+template <int MODE, int KMAX>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const Params p) {
@@ -109,6 +116,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   int* fill_par = reinterpret_cast<int*>(tmem_slot + 2);  // [STAGES]
   int* s_off = fill_par + STAGES;                          // [G+1]
   int* s_cum = s_off + (p.G + 1);                          // [G+1]
+  float* s_bias = reinterpret_cast<float*>(s_cum + (p.G + 1));  // [E], router only
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int G = p.G;
@@ -133,6 +141,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
+  if (MODE == MODE_ROUTER)
+    for (int e = threadIdx.x; e < p.E; e += THREADS) s_bias[e] = p.bias ? p.bias[e] : 0.f;
   if (p.offsets) {
     for (int g = threadIdx.x; g <= G; g += THREADS) s_off[g] = p.offsets[g];
   } else if (threadIdx.x == 0) {
@@ -182,7 +192,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             break;
           }
           const uint32_t fb = smem_u32(&full[stage]);
-          mbar_expect_tx(fb, A_BYTES + B_BYTES);
+          mbar_expect_tx(fb, A_BYTES + (MODE == MODE_ROUTER ? p.n_mma * BK * 2 : B_BYTES));
           fill_par[stage] = (int)phase;
           tma_load_2d(smem_u32(sA + stage * A_BYTES), &tmA, fb, kb * BK, a_row);
           if (MODE == MODE_SWIGLU) {
@@ -202,7 +212,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN_MMA);
+      const uint32_t idesc = idesc_bf16_f32(BM, MODE == MODE_ROUTER ? p.n_mma : BN_MMA);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -277,6 +287,62 @@ __global__ void __launch_bounds__(THREADS, 1)
             } else {
               const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(pk);
               for (int j = 0; j < 32 && col_base + c + j < p.N; ++j) orow[c + j] = hv[j];
+            }
+          }
+        }
+      } else if (MODE == MODE_ROUTER) {
+        // Keep the top k of kappa = logit + bias over the E columns of this row,
+        // then the gate weights of the chosen experts.
+        TopK<KMAX> tk;
+        tk.init();
+        float mx = -INFINITY;
+        const int E = p.E;
+#pragma unroll 1
+        for (int c = 0; c < p.n_mma; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(tb + c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (c + j < E) {
+              const float l = __uint_as_float(v[j]);
+              const float kap = l + s_bias[c + j];
+              tk.push(kap, c + j, l);
+              mx = fmaxf(mx, kap);
+            }
+          }
+        }
+        float z = 0.f;
+        if (p.gating == 0) {  // softmax over all E: needs the full denominator
+#pragma unroll 1
+          for (int c = 0; c < p.n_mma; c += 32) {
+            uint32_t v[32];
+            tmem_ld32(tb + c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c + j < E) z += expf(__uint_as_float(v[j]) + s_bias[c + j] - mx);
+          }
+        }
+        if (ok) {
+          float wsel[KMAX];
+          float den = 0.f;
+#pragma unroll
+          for (int s = 0; s < KMAX; ++s) {
+            float wv = 0.f;
+            if (s < p.k) {
+              if (p.gating == 0) wv = expf(tk.key[s] - mx) / z;
+              else if (p.gating == 1) wv = expf(tk.key[s] - tk.key[0]);
+              else wv = 1.0f / (1.0f + expf(-(p.bias_select_only ? tk.val[s] : tk.key[s])));
+            }
+            wsel[s] = wv;
+            den += wv;
+          }
+#pragma unroll
+          for (int s = 0; s < KMAX; ++s) {
+            if (s < p.k) {
+              p.ids[grow * p.k + s] = tk.idx[s];
+              p.wts[grow * p.k + s] = wsel[s] / den;
             }
           }
         }
@@ -356,17 +422,17 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE>
+template <int MODE, int KMAX>
 cudaError_t launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, int64_t tiles_bound,
                         cudaStream_t stream) {
-  const size_t smem = smem_bytes(p.G);
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  const size_t smem = smem_bytes(p.G, MODE == MODE_ROUTER ? p.E : 0);
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<MODE, KMAX>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int64_t grid = device_sm_count();
   if (tiles_bound < grid) grid = tiles_bound;
   if (grid < 1) grid = 1;
-  grouped_gemm_tc_kernel<MODE><<<(unsigned)grid, THREADS, smem, stream>>>(ta, tb, p);
+  grouped_gemm_tc_kernel<MODE, KMAX><<<(unsigned)grid, THREADS, smem, stream>>>(ta, tb, p);
   return cudaGetLastError();
 }
 
@@ -384,12 +450,32 @@ cudaError_t launch_grouped_ffn_bf16_tc(const GroupedFfnArgs& a, cudaStream_t str
   const int64_t mt_bound = (a.rows + BM - 1) / BM + (a.offsets ? a.G : 0);
   const uint64_t lim = a.wait_limit_ns ? a.wait_limit_ns : 2000000000ull;
   Params p1{a.offsets, G, a.rows, a.d, a.f, (a.f + bn_out(MODE_SWIGLU) - 1) / bn_out(MODE_SWIGLU),
-            2 * (int64_t)a.f, a.f, a.h, a.f, a.status, lim};
-  cudaError_t e = launch_mode<MODE_SWIGLU>(mA1, mB1, p1, mt_bound * p1.nt, stream);
+            2 * (int64_t)a.f, a.f, a.h, a.f, a.status, lim, BN_MMA};
+  cudaError_t e = launch_mode<MODE_SWIGLU, 1>(mA1, mB1, p1, mt_bound * p1.nt, stream);
   if (e != cudaSuccess) return e;
   Params p2{a.offsets, G, a.rows, a.f, a.d, (a.d + bn_out(MODE_PLAIN) - 1) / bn_out(MODE_PLAIN), (int64_t)a.d, 0,
-            a.y, a.d, a.status, lim};
-  return launch_mode<MODE_PLAIN>(mA2, mB2, p2, mt_bound * p2.nt, stream);
+            a.y, a.d, a.status, lim, BN_MMA};
+  return launch_mode<MODE_PLAIN, 1>(mA2, mB2, p2, mt_bound * p2.nt, stream);
+}
+
+// Router GEMM on the tensor cores with the top-k and gate weights fused into
+// the epilogue: one 128-token tile per CTA, N = E rounded up to 16 (the rows of
+// W_r past E are zero-filled by the TMA box and never selected).
+cudaError_t launch_router_topk_tc(const RouterArgs& a, cudaStream_t stream) {
+  using namespace tc;
+  if (!a.bf16 || a.E > BN_MMA || a.k > 16) return cudaErrorInvalidValue;
+  const int n_mma = ((a.E + 15) / 16) * 16;
+  CUtensorMap mA, mB;
+  if (!make_map(&mA, a.x, (uint64_t)a.T, a.d, BM) || !make_map(&mB, a.w_router, (uint64_t)a.E, a.d, n_mma))
+    return cudaErrorInvalidValue;
+  const uint64_t lim = a.wait_limit_ns ? a.wait_limit_ns : 2000000000ull;
+  Params p{nullptr, 1, a.T, a.d, a.E, 1, 0, 0, nullptr, 0, a.status, lim, n_mma,
+           a.bias, a.ids, a.w, a.E, a.k, a.gating, a.bias_select_only};
+  const int64_t tiles = (a.T + BM - 1) / BM;
+  if (a.k <= 2) return launch_mode<MODE_ROUTER, 2>(mA, mB, p, tiles, stream);
+  if (a.k <= 4) return launch_mode<MODE_ROUTER, 4>(mA, mB, p, tiles, stream);
+  if (a.k <= 8) return launch_mode<MODE_ROUTER, 8>(mA, mB, p, tiles, stream);
+  return launch_mode<MODE_ROUTER, 16>(mA, mB, p, tiles, stream);
 }
 
 }  // namespace moe

@@ -21,7 +21,9 @@ struct RouterArgs {
   int* status;
   uint64_t wait_limit_ns;
 };
-cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t stream);
+cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t stream);       // picks one of:
+cudaError_t launch_router_topk_simt(const RouterArgs& a, cudaStream_t stream);  // CUDA cores, any dtype
+cudaError_t launch_router_topk_tc(const RouterArgs& a, cudaStream_t stream);    // tcgen05, bf16, E <= 256
 
 // ---- dispatch (permute.cu)
 struct PermuteArgs {

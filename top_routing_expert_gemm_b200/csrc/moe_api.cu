@@ -16,9 +16,13 @@ int device_sm_count() {
   return n;
 }
 
-cudaError_t launch_router_topk_simt(const RouterArgs& a, cudaStream_t stream);
-
+// Router kernel choice: with many experts the router is a real GEMM
+// (2*T*d*E flops: 30 GFLOP for T=8192, d=7168, E=256) and runs on the tensor
+// cores with the top-k fused into the epilogue; with few experts (or fp32,
+// which must not use TF32) W_r fits in shared memory and a warp per token on
+// the CUDA cores is cheaper than a 128-token tensor tile.
 cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t stream) {
+  if (a.bf16 && a.E >= 64 && a.E <= 256) return launch_router_topk_tc(a, stream);
   return launch_router_topk_simt(a, stream);
 }
 
@@ -222,6 +226,13 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
   moe_status st = check_config(cfg);
   if (st != MOE_OK) return st;
   if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+  if (cfg->T == 0) {  // nothing to read or write: clear the status word and the optional counts
+    if (opt_counts && !aligned16(opt_counts)) return MOE_ERR_INVALID_ARG;
+    if ((st = bind(ws)) != MOE_OK) return st;
+    MOE_CUDA_TRY(cudaMemsetAsync(ws, 0, 16, stream));
+    if (opt_counts) MOE_CUDA_TRY(cudaMemsetAsync(opt_counts, 0, sizeof(int32_t) * cfg->n_experts, stream));
+    return MOE_OK;
+  }
   if (!x || !w_router || !w_gate_up || !w_down || !y || !aligned16(x) || !aligned16(w_router) ||
       !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(y) || (logit_bias && !aligned16(logit_bias)) ||
       (opt_topk_ids && !aligned16(opt_topk_ids)) || (opt_topk_w && !aligned16(opt_topk_w)) ||
@@ -236,10 +247,6 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
   int32_t* ids = opt_topk_ids ? opt_topk_ids : k.ids;
   float* w = opt_topk_w ? opt_topk_w : k.w;
   int32_t* counts = opt_counts ? opt_counts : k.counts;
-  if (cfg->T == 0) {
-    MOE_CUDA_TRY(cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->n_experts, stream));
-    return MOE_OK;
-  }
   RouterArgs ra{x, w_router, logit_bias, ids, w, cfg->T, cfg->d_model, cfg->n_experts, cfg->top_k,
                 cfg->gating, cfg->bias_select_only, cfg->dtype == MOE_BF16, k.status, wait_limit(cfg)};
   MOE_CUDA_TRY(launch_router_topk(ra, stream));

@@ -46,23 +46,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase of `parity` to complete, for at most `limit_ns`.  Gives
-// up early when another role of the CTA has raised `abort`.  Returns false
-// (after raising `abort` and the device status word on a timeout) when the
-// phase did not complete.
+// Wait for the phase of `parity` to complete, for at most `limit_ns`.  Each
+// try_wait may suspend the thread for a hardware-defined slice; after every
+// slice that ends without completion the abort flag and the clock are checked.
+// Gives up early when another role of the CTA has raised `abort`.  Returns
+// false (after raising `abort` and the device status word on a timeout) when
+// the phase did not complete.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort,
                                                   uint64_t limit_ns, int* status) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
+  while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 15u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
-        *abort = 1;
-        set_status(status, kDevTimeout);
-        return false;
-      }
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort = 1;
+      set_status(status, kDevTimeout);
+      return false;
     }
   }
 }
