@@ -61,8 +61,7 @@ __global__ void __launch_bounds__(kThreads) router_topk_simt_kernel(RouterParams
       float acc[kGroup];
 #pragma unroll
       for (int j = 0; j < kGroup; ++j) acc[j] = 0.f;
-      for (int i0 = lane * V; i0 < d; i0 += 32 * V) {
-        const Vec16<T> xv = ld16(xr + i0);
+      auto fma_chunk = [&](const Vec16<T>& xv, int i0) {
         float xf[V];
 #pragma unroll
         for (int v = 0; v < V; ++v) xf[v] = Elem<T>::to_f(xv.v[v]);
@@ -77,7 +76,17 @@ __global__ void __launch_bounds__(kThreads) router_topk_simt_kernel(RouterParams
             for (int v = 0; v < V; ++v) acc[j] = fmaf(xf[v], Elem<T>::to_f(wv.v[v]), acc[j]);
           }
         }
+      };
+      // four row chunks in flight per lane: the x row streams from HBM
+      int i0 = lane * V;
+      for (; i0 + 3 * 32 * V < d; i0 += 4 * 32 * V) {
+        Vec16<T> xv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) xv[u] = ld16(xr + i0 + u * 32 * V);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) fma_chunk(xv[u], i0 + u * 32 * V);
       }
+      for (; i0 < d; i0 += 32 * V) fma_chunk(ld16(xr + i0), i0);
 #pragma unroll
       for (int j = 0; j < kGroup; ++j)
 #pragma unroll
