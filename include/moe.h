@@ -138,6 +138,29 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_ids, const voi
                        int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* row_of,
                        void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_permute without a workspace.  No counterpart on the pages: this is a
+   calling convention for callers that cannot provide device scratch when they
+   dispatch -- e.g. a plug-in whose host framework owns every device
+   allocation and passes it only tensors, or a serving loop whose memory policy
+   forbids allocating once it runs (an allocation there may stall the device,
+   or fail with out-of-memory in the middle of a step).
+   Same arguments and results as moe_permute, minus ws/ws_bytes.  The
+   per-(expert, chunk) histogram lives in a 256 KiB array compiled into the
+   library (held on every GPU that loads it until the process exits):
+   n_experts * ceil(T*k / 2048) must be <= 65536, else MOE_ERR_UNSUPPORTED and
+   nothing runs; an invalid config returns MOE_ERR_INVALID_ARG.  The call
+   allocates nothing.  The first call on a device looks up the array's device
+   address (with that device current) and keeps it for the rest of the process;
+   make that first call before any stream capture, and do not reset the device
+   afterwards.  All calls share the one array: calls that overlap on the GPU
+   (different streams, or several host threads) race and must be serialised by
+   the caller.  Every call rewrites the part of the array it reads, so nothing
+   has to be cleared between calls.  There is no status word: an id outside
+   [0, E) is skipped (its row_of is -1) and is not reported. */
+moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* topk_ids, const void* x,
+                               int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* row_of,
+                               void* x_perm, moe_stream_t stream);
+
 /* Grouped SwiGLU experts over the dispatched rows.
    x_perm [T*k, d], offsets [E+1] (device), w_gate_up [E, 2f, d] (rows 0..f-1
    gate, f..2f-1 up), w_down [E, d, f] -> y_perm [T*k, d].

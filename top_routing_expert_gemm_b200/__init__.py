@@ -13,6 +13,7 @@ import pathlib
 __all__ = [
     "MoeError", "MoeConfig", "lib", "make_config", "moe_workspace_bytes", "moe_status_string",
     "moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_forward", "moe_device_status",
+    "moe_permute_noalloc",
     "MOE_F32", "MOE_BF16", "MOE_SOFTMAX_ALL_RENORM", "MOE_SOFTMAX_TOPK", "MOE_SIGMOID_TOPK_RENORM",
     "EXPORTED_SYMBOLS", "LIB_PATH",
 ]
@@ -27,7 +28,7 @@ MOE_SOFTMAX_ALL_RENORM, MOE_SOFTMAX_TOPK, MOE_SIGMOID_TOPK_RENORM = 0, 1, 2
 
 EXPORTED_SYMBOLS = (
     "moe_workspace_bytes", "moe_status_string", "moe_router_topk", "moe_permute", "moe_grouped_ffn",
-    "moe_combine", "moe_forward", "moe_device_status",
+    "moe_combine", "moe_forward", "moe_device_status", "moe_permute_noalloc",
 )
 
 
@@ -76,6 +77,7 @@ def lib() -> ctypes.CDLL:
         L.moe_combine.argtypes = [cfgp, vp, vp, vp, vp, vp, vp]
         L.moe_forward.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_device_status.argtypes = [vp, sz, vp]
+        L.moe_permute_noalloc.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp]
         for name in EXPORTED_SYMBOLS[2:]:
             getattr(L, name).restype = i32
         _lib = L
@@ -130,6 +132,12 @@ def moe_permute(cfg, topk_ids, x, counts, offsets, perm, row_of, x_perm, ws, ws_
     nb = ws_bytes if ws_bytes is not None else ws.numel() * ws.element_size()
     _check(lib().moe_permute(ctypes.byref(cfg), _p(topk_ids), _p(x), _p(counts), _p(offsets), _p(perm),
                              _p(row_of), _p(x_perm), _p(ws), nb, _stream(stream)), "moe_permute")
+
+
+def moe_permute_noalloc(cfg, topk_ids, x, counts, offsets, perm, row_of, x_perm, stream=None) -> None:
+    """moe_permute without a workspace (its scratch is a fixed array inside the library)."""
+    _check(lib().moe_permute_noalloc(ctypes.byref(cfg), _p(topk_ids), _p(x), _p(counts), _p(offsets), _p(perm),
+                                     _p(row_of), _p(x_perm), _stream(stream)), "moe_permute_noalloc")
 
 
 def moe_grouped_ffn(cfg, x_perm, offsets, w_gate_up, w_down, y_perm, ws, ws_bytes=None, stream=None) -> None:
