@@ -7,16 +7,19 @@
 // VRAM" (a gated feed-forward block with three matrices), read as SwiGLU.
 //
 //   GEMM-1 (MODE_SWIGLU): h[rows, f] = SiLU(A Wg^T) * (A Wu^T), one launch
-//     over every expert; each 128x256 accumulator holds 128 gate columns and
-//     the matching 128 up columns, so the SwiGLU is applied in the epilogue
-//     straight out of tensor memory and only h (bf16) reaches HBM.
+//     over every expert; each 128 x N accumulator holds N/2 gate columns and
+//     the matching N/2 up columns (the B tile is the gate rows followed by the
+//     up rows), so the SwiGLU is applied in the epilogue straight out of
+//     tensor memory and only h (bf16) reaches HBM.
 //   GEMM-2 (MODE_PLAIN):  y[rows, d] = h Wd^T.
+//   Router (MODE_ROUTER): logits = x W_r^T with N = E rounded up to 16; the
+//     epilogue keeps the top k per row and writes ids and gate weights.
 //
 // Persistent, warp-specialised CTA (192 threads, one CTA per SM):
-//   warp 0     TMA producer: 4-stage ring of (A 128x64, B 256x64) bf16 tiles,
+//   warp 0     TMA producer: 4-stage ring of (A 128x64, B Nx64) bf16 tiles,
 //              128-byte swizzle, mbarrier transaction counts
 //   warp 1     TMEM allocator and single-thread tcgen05.mma issuer
-//              (M=128, N=256, K=16 per instruction, fp32 accumulators)
+//              (M=128, N<=256, K=16 per instruction, fp32 accumulators)
 //   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter, SwiGLU / bf16
 //              conversion, masked 16-byte stores
 // Two 256-column accumulators (all 512 TMEM columns) let the epilogue of tile
@@ -68,8 +71,6 @@ struct Params {
   float* wts;              // [rows, k]
   int E, k, gating, bias_select_only;
 };
-
-__host__ __device__ constexpr int bn_out(int mode) { return mode == MODE_SWIGLU ? BN_MMA / 2 : BN_MMA; }
 
 size_t smem_bytes(int G, int E) {
   return 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + 256 + 2 * sizeof(int) * (size_t)(G + 1) +
@@ -173,7 +174,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int64_t total = (int64_t)s_cum[G] * p.nt;
   const int kb_count = (p.K + BK - 1) / BK;
-  constexpr int BNO = bn_out(MODE);
+  const int n_mma = p.n_mma;
+  const int bno = MODE == MODE_SWIGLU ? n_mma / 2 : n_mma;  // output columns per tile
 
   if (warp == 0) {
     if (lane == 0) {
@@ -184,7 +186,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         int g, mt, ntile;
         decode_tile(t, p.nt, s_cum, G, g, mt, ntile);
         const int a_row = s_off[g] + mt * BM;
-        const int b_row = (int)((int64_t)g * p.b_group_rows + (int64_t)ntile * BNO);
+        const int b_row = (int)((int64_t)g * p.b_group_rows + (int64_t)ntile * bno);
         bool ok = true;
         for (int kb = 0; kb < kb_count; ++kb) {
           if (!mbar_wait_bounded(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, p.wait_limit_ns, p.status)) {
@@ -192,12 +194,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             break;
           }
           const uint32_t fb = smem_u32(&full[stage]);
-          mbar_expect_tx(fb, A_BYTES + (MODE == MODE_ROUTER ? p.n_mma * BK * 2 : B_BYTES));
+          mbar_expect_tx(fb, A_BYTES + n_mma * BK * 2);
           fill_par[stage] = (int)phase;
           tma_load_2d(smem_u32(sA + stage * A_BYTES), &tmA, fb, kb * BK, a_row);
-          if (MODE == MODE_SWIGLU) {
+          if (MODE == MODE_SWIGLU) {  // gate rows, then the matching up rows (bno is a multiple of 8)
             tma_load_2d(smem_u32(sB + stage * B_BYTES), &tmB, fb, kb * BK, b_row);
-            tma_load_2d(smem_u32(sB + stage * B_BYTES + B_BYTES / 2), &tmB, fb, kb * BK, b_row + p.up_off);
+            tma_load_2d(smem_u32(sB + stage * B_BYTES + bno * BK * 2), &tmB, fb, kb * BK, b_row + p.up_off);
           } else {
             tma_load_2d(smem_u32(sB + stage * B_BYTES), &tmB, fb, kb * BK, b_row);
           }
@@ -212,7 +214,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      const uint32_t idesc = idesc_bf16_f32(BM, MODE == MODE_ROUTER ? p.n_mma : BN_MMA);
+      const uint32_t idesc = idesc_bf16_f32(BM, n_mma);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -263,34 +265,44 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int64_t grow = (int64_t)s_off[g] + lr;
       const bool ok = lr < rows_g && grow >= 0 && grow < p.rows;
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MMA);
-      const int col_base = ntile * BNO;
+      const int col_base = ntile * bno;
+      const int col_lim = min(p.N, col_base + bno);  // this tile's columns (bno need not be a multiple of 32)
       __nv_bfloat16* orow = out + grow * p.ldo + col_base;
-      if (MODE == MODE_SWIGLU) {
+      if (MODE != MODE_ROUTER) {
+        // SwiGLU mode: gate in accumulator columns [0, bno), up in [bno, 2 bno);
+        // plain mode: the bno output columns
 #pragma unroll 1
-        for (int c = 0; c < BNO; c += 32) {
-          uint32_t gv[32], uv[32];
-          tmem_ld32(tb + c, gv);
-          tmem_ld32(tb + BNO + c, uv);
+        for (int c = 0; c < bno; c += 32) {
+          uint32_t v[32], u[32];
+          tmem_ld32(tb + c, v);
+          if (MODE == MODE_SWIGLU) tmem_ld32(tb + bno + c, u);
           tmem_ld_wait();
           if (ok) {
             uint32_t pk[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              const float h0 = silu_f(__uint_as_float(gv[2 * j])) * __uint_as_float(uv[2 * j]);
-              const float h1 = silu_f(__uint_as_float(gv[2 * j + 1])) * __uint_as_float(uv[2 * j + 1]);
+              float h0 = __uint_as_float(v[2 * j]), h1 = __uint_as_float(v[2 * j + 1]);
+              if (MODE == MODE_SWIGLU) {
+                h0 = silu_f(h0) * __uint_as_float(u[2 * j]);
+                h1 = silu_f(h1) * __uint_as_float(u[2 * j + 1]);
+              }
               pk[j] = pack_bf16x2(h0, h1);
             }
-            if (col_base + c + 32 <= p.N) {
+            if (col_base + c + 32 <= col_lim) {
               uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
               for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
             } else {
-              const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(pk);
-              for (int j = 0; j < 32 && col_base + c + j < p.N; ++j) orow[c + j] = hv[j];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const int cc = col_base + c + 2 * j;
+                if (cc < col_lim) orow[c + 2 * j] = __ushort_as_bfloat16((unsigned short)(pk[j] & 0xFFFFu));
+                if (cc + 1 < col_lim) orow[c + 2 * j + 1] = __ushort_as_bfloat16((unsigned short)(pk[j] >> 16));
+              }
             }
           }
         }
-      } else if (MODE == MODE_ROUTER) {
+      } else {
         // Keep the top k of kappa = logit + bias over the E columns of this row,
         // then the gate weights of the chosen experts.
         TopK<KMAX> tk;
@@ -346,26 +358,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
           }
         }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < BNO; c += 32) {
-          uint32_t v[32];
-          tmem_ld32(tb + c, v);
-          tmem_ld_wait();
-          if (ok) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-            if (col_base + c + 32 <= p.N) {
-              uint4* dst = reinterpret_cast<uint4*>(orow + c);
-#pragma unroll
-              for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-            } else {
-              const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(pk);
-              for (int j = 0; j < 32 && col_base + c + j < p.N; ++j) orow[c + j] = hv[j];
-            }
-          }
-        }
       }
       tc_fence_before();
       mbar_arrive(smem_u32(&tempty[acc]));
@@ -374,6 +366,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   }
 
+  if (warp == 0 && lane == 0 && !*abort_flag) {
+    // every stage filled has been released by its MMAs (their completion
+    // arrivals target this CTA's barriers, which must outlive them)
+    for (int s = 0; s < STAGES; ++s)
+      if (fill_par[s] >= 0) drain_wait(smem_u32(&empty[s]), (uint32_t)fill_par[s]);
+  }
   __syncthreads();
   if (*abort_flag) {
     // let this CTA's own asynchronous copies and MMAs land before its shared
@@ -442,19 +440,25 @@ cudaError_t launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const Para
 cudaError_t launch_grouped_ffn_bf16_tc(const GroupedFfnArgs& a, cudaStream_t stream) {
   using namespace tc;
   if (a.rows == 0) return cudaSuccess;
-  CUtensorMap mA1, mB1, mA2, mB2;
-  if (!make_map(&mA1, a.a, a.rows, a.d, BM) || !make_map(&mB1, a.w_gate_up, (uint64_t)a.G * 2 * a.f, a.d, BN_MMA / 2) ||
-      !make_map(&mA2, a.h, a.rows, a.f, BM) || !make_map(&mB2, a.w_down, (uint64_t)a.G * a.d, a.f, BN_MMA))
-    return cudaErrorInvalidValue;
   const int G = a.offsets ? a.G : 1;
   const int64_t mt_bound = (a.rows + BM - 1) / BM + (a.offsets ? a.G : 0);
   const uint64_t lim = a.wait_limit_ns ? a.wait_limit_ns : 2000000000ull;
-  Params p1{a.offsets, G, a.rows, a.d, a.f, (a.f + bn_out(MODE_SWIGLU) - 1) / bn_out(MODE_SWIGLU),
-            2 * (int64_t)a.f, a.f, a.h, a.f, a.status, lim, BN_MMA};
+  // GEMM-1 + SwiGLU: tile = 128 rows x (128 gate + 128 up) columns.  Narrower
+  // or non-power-of-two MMA widths measured slower on the layer shapes here.
+  const int n1 = BN_MMA;
+  CUtensorMap mA1, mB1;
+  if (!make_map(&mA1, a.a, a.rows, a.d, BM) || !make_map(&mB1, a.w_gate_up, (uint64_t)a.G * 2 * a.f, a.d, n1 / 2))
+    return cudaErrorInvalidValue;
+  Params p1{a.offsets, G, a.rows, a.d, a.f, (a.f + n1 / 2 - 1) / (n1 / 2), 2 * (int64_t)a.f, a.f, a.h, a.f,
+            a.status, lim, n1};
   cudaError_t e = launch_mode<MODE_SWIGLU, 1>(mA1, mB1, p1, mt_bound * p1.nt, stream);
   if (e != cudaSuccess) return e;
-  Params p2{a.offsets, G, a.rows, a.f, a.d, (a.d + bn_out(MODE_PLAIN) - 1) / bn_out(MODE_PLAIN), (int64_t)a.d, 0,
-            a.y, a.d, a.status, lim, BN_MMA};
+  // GEMM-2: tile = 128 rows x 256 output columns
+  const int n2 = BN_MMA;
+  CUtensorMap mA2, mB2;
+  if (!make_map(&mA2, a.h, a.rows, a.f, BM) || !make_map(&mB2, a.w_down, (uint64_t)a.G * a.d, a.f, n2))
+    return cudaErrorInvalidValue;
+  Params p2{a.offsets, G, a.rows, a.f, a.d, (a.d + n2 - 1) / n2, (int64_t)a.d, 0, a.y, a.d, a.status, lim, n2};
   return launch_mode<MODE_PLAIN, 1>(mA2, mB2, p2, mt_bound * p2.nt, stream);
 }
 
