@@ -77,7 +77,7 @@ def test_host_checks_reject_before_launch(L):
     assert _call_forward(L, _cfg(top_k=17, n_experts=32)) == 2      # beyond the build's limits
     assert _call_forward(L, _cfg(), ws_bytes=16) == 3               # workspace too small
     assert _call_forward(L, _cfg(), ptr=258) == 1                   # misaligned pointers
-    assert _call_forward(L, _cfg(n_shared=1, d_ff_shared=512)) == 1  # shared weights missing
+    assert _call_forward(L, _cfg(n_shared=1, d_ff_shared=512), ws_bytes=1 << 30) == 1  # shared weights missing
     cfg = _cfg()
     assert L.moe_forward(ctypes.byref(cfg), None, None, None, None, None, None, None, None, None, None, None,
                          ctypes.c_void_p(256), 1 << 30, None) == 1  # null tensors

@@ -177,6 +177,8 @@ def _ragged_offsets(sizes):
     ([5, 0, 140], 264, 200),                     # partial n-tiles in both GEMMs
     ([1000], 512, 1024),                          # one big group
     ([3] * 40, 128, 136),                         # many tiny groups
+    ([70, 0, 1, 64, 65], 4096, 640),              # decode kernel: 2-chunk groups, split-K GEMM-1
+    ([1, 1], 4096, 14336),                        # decode kernel: one token per expert, split-K GEMM-2
 ])
 def test_grouped_ffn_against_dense_experts(dtype, sizes, d, f):
     rng = np.random.default_rng(sum(sizes) + d + f)

@@ -57,9 +57,19 @@ struct GroupedFfnArgs {
   int G, d, f;
   int* status;
   uint64_t wait_limit_ns;
+  // decode kernel only: split-K partial tiles and per-tile arrival counters
+  float* partial;
+  int64_t partial_slots;
+  int* counters;
+  int64_t counter_cap;
 };
-cudaError_t launch_grouped_ffn_bf16_tc(const GroupedFfnArgs& a, cudaStream_t stream);  // tcgen05
-cudaError_t launch_grouped_ffn_f32_simt(const GroupedFfnArgs& a, cudaStream_t stream);  // fp32 CUDA cores
+cudaError_t launch_grouped_ffn_bf16_tc(const GroupedFfnArgs& a, cudaStream_t stream);      // tcgen05, large batch
+cudaError_t launch_grouped_ffn_bf16_decode(const GroupedFfnArgs& a, cudaStream_t stream);  // tcgen05, swap-AB
+cudaError_t launch_grouped_ffn_f32_simt(const GroupedFfnArgs& a, cudaStream_t stream);      // fp32 CUDA cores
+// decode regime: at most 64 rows per touched group on average (uniform-routing expectation)
+bool use_decode_ffn(int64_t rows, int G, bool grouped);
+int64_t decode_partial_slots(int64_t rows, int G, bool grouped, int d, int f);
+int64_t decode_counter_cap(int64_t rows, int G, int d, int f);
 
 // ---- combine (combine.cu)
 struct CombineArgs {

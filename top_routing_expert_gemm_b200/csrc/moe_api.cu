@@ -3,6 +3,8 @@
 // allocates device memory or synchronises, except moe_device_status.
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "../../include/moe.h"
 #include "common.cuh"
 #include "kernels.cuh"
@@ -60,8 +62,20 @@ struct Carve {
   int32_t *ids, *counts, *offsets, *perm, *row_of, *chunk_counts;
   float* w;
   void *x_perm, *h, *y_perm, *h_s, *y_s;
+  float* partial;           // decode split-K partial tiles (bf16 decode regime only)
+  int64_t partial_slots;
+  int* counters;
+  int64_t counter_cap;
   size_t total;
 };
+
+// Does this config run its routed / shared experts on the decode kernel?
+bool decode_routed(const moe_config* c) {
+  return c->dtype == MOE_BF16 && use_decode_ffn(c->T * c->top_k, c->n_experts, true);
+}
+bool decode_shared(const moe_config* c) {
+  return c->dtype == MOE_BF16 && c->n_shared > 0 && use_decode_ffn(c->T, 1, false);
+}
 
 // Lay out the workspace; with base == nullptr only sizes are computed.
 Carve carve(const moe_config* c, void* base) {
@@ -89,6 +103,13 @@ Carve carve(const moe_config* c, void* base) {
   if (c->n_shared > 0) {
     k.h_s = take(eb * c->T * c->d_ff_shared);
     k.y_s = take(eb * c->T * c->d_model);
+  }
+  if (decode_routed(c) || decode_shared(c)) {
+    k.partial_slots = decode_partial_slots(n, c->n_experts, true, c->d_model, c->d_ff);
+    k.partial = static_cast<float*>(take(sizeof(float) * 128 * 64 * (size_t)k.partial_slots));
+    k.counter_cap = std::max(decode_counter_cap(n, c->n_experts, c->d_model, c->d_ff),
+                             c->n_shared ? decode_counter_cap(c->T, 1, c->d_model, c->d_ff_shared) : 0);
+    k.counters = static_cast<int*>(take(sizeof(int) * (size_t)k.counter_cap));
   }
   k.total = off;
   return k;
@@ -123,10 +144,13 @@ moe_status bind(const void* p) {
 
 uint64_t wait_limit(const moe_config* c) { return c->wait_limit_ns > 0 ? (uint64_t)c->wait_limit_ns : 2000000000ull; }
 
-cudaError_t run_ffn(const moe_config* c, const void* a, const int32_t* offsets, int G, int64_t rows, int f,
-                    const void* w_gu, const void* w_d, void* h, void* y, int* status, cudaStream_t s) {
-  GroupedFfnArgs g{a, offsets, w_gu, w_d, h, y, rows, G, c->d_model, f, status, wait_limit(c)};
-  return c->dtype == MOE_BF16 ? launch_grouped_ffn_bf16_tc(g, s) : launch_grouped_ffn_f32_simt(g, s);
+cudaError_t run_ffn(const moe_config* c, const Carve& k, const void* a, const int32_t* offsets, int G, int64_t rows,
+                    int f, const void* w_gu, const void* w_d, void* h, void* y, cudaStream_t s) {
+  GroupedFfnArgs g{a, offsets, w_gu, w_d, h, y, rows, G, c->d_model, f, k.status, wait_limit(c),
+                   k.partial, k.partial_slots, k.counters, k.counter_cap};
+  if (c->dtype != MOE_BF16) return launch_grouped_ffn_f32_simt(g, s);
+  if (k.partial != nullptr && use_decode_ffn(rows, G, offsets != nullptr)) return launch_grouped_ffn_bf16_decode(g, s);
+  return launch_grouped_ffn_bf16_tc(g, s);
 }
 
 }  // namespace
@@ -200,8 +224,8 @@ moe_status moe_grouped_ffn(const moe_config* cfg, const void* x_perm, const int3
     return MOE_ERR_INVALID_ARG;
   if ((st = bind(ws)) != MOE_OK) return st;
   Carve k = carve(cfg, ws);
-  MOE_CUDA_TRY(run_ffn(cfg, x_perm, offsets, cfg->n_experts, cfg->T * cfg->top_k, cfg->d_ff, w_gate_up, w_down,
-                       k.h, y_perm, k.status, stream));
+  MOE_CUDA_TRY(run_ffn(cfg, k, x_perm, offsets, cfg->n_experts, cfg->T * cfg->top_k, cfg->d_ff, w_gate_up, w_down,
+                       k.h, y_perm, stream));
   return MOE_OK;
 }
 
@@ -253,11 +277,10 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
   PermuteArgs pa{ids, x, counts, k.offsets, k.perm, k.row_of, k.x_perm, k.chunk_counts, cfg->T * cfg->top_k,
                  cfg->top_k, cfg->d_model, cfg->n_experts, (int)elem_bytes(cfg), k.status};
   MOE_CUDA_TRY(launch_permute(pa, stream));
-  MOE_CUDA_TRY(run_ffn(cfg, k.x_perm, k.offsets, cfg->n_experts, cfg->T * cfg->top_k, cfg->d_ff, w_gate_up, w_down,
-                       k.h, k.y_perm, k.status, stream));
+  MOE_CUDA_TRY(run_ffn(cfg, k, k.x_perm, k.offsets, cfg->n_experts, cfg->T * cfg->top_k, cfg->d_ff, w_gate_up,
+                       w_down, k.h, k.y_perm, stream));
   if (cfg->n_shared > 0)
-    MOE_CUDA_TRY(run_ffn(cfg, x, nullptr, 1, cfg->T, cfg->d_ff_shared, ws_gate_up, ws_down, k.h_s, k.y_s, k.status,
-                         stream));
+    MOE_CUDA_TRY(run_ffn(cfg, k, x, nullptr, 1, cfg->T, cfg->d_ff_shared, ws_gate_up, ws_down, k.h_s, k.y_s, stream));
   CombineArgs ca{k.y_perm, k.row_of, w, cfg->n_shared > 0 ? k.y_s : nullptr, y, cfg->T, cfg->top_k,
                  cfg->d_model, cfg->dtype == MOE_BF16};
   MOE_CUDA_TRY(launch_combine(ca, stream));
