@@ -10,7 +10,7 @@ the CUDA path; the only common dependency is the seeded input generator
 Everything is float64 numpy.  Stored inputs (float32 or bfloat16 values) are
 upcast exactly, then the layer is evaluated with no intermediate rounding.
 Library primitives used as single steps: ``@`` (matrix product), ``np.exp``,
-``np.argsort(kind="stable")``.
+``np.log``, ``scipy.special.erf``, ``np.argsort(kind="stable")``.
 
 Sources (page title, then section):
 
@@ -47,8 +47,19 @@ Readings where the pages are silent (each also listed in the design notes):
   weights); the sigmoid rule with ``bias_select_only`` uses it for
   selection only ([AFD] "Why load balancing...": the bias shifts routing
   without distorting the gate values used for output).
-* The output is the MoE sublayer alone (no residual), dropless, and shared
-  experts enter with weight 1.
+* The output is the MoE sublayer alone (no residual), dropless unless a
+  capacity is given, and shared experts enter with weight 1.
+* Capacity: ceil(T*k/E * factor) rows per expert ([SEV]'s script counts
+  routing slots); an expert keeps its first arrivals in token order (the
+  pages say only that tokens "beyond that limit" skip the expert); a dropped
+  slot adds nothing and the token's other weights are not rescaled.
+* Balance loss and z-loss are computed from the bias-free router logits
+  (the pages define them on the router's own output) and returned without
+  their loss weights (alpha = 0.01, 0.001 on the pages); the balance loss
+  counts routing slots before any capacity cut, and the z-loss is the mean
+  over tokens of the squared log-sum-exp.
+* Two-matrix expert: [SEV]'s build, ``GELU(x W_up^T) W_down^T`` with the exact
+  (erf) GELU, its library default.
 
 Parity is pinned by ``tests/test_oracle_pins.py`` against closed forms, the
 pages' printed numbers and brute force; see each function's docstring.
@@ -56,6 +67,7 @@ pages' printed numbers and brute force; see each function's docstring.
 from __future__ import annotations
 
 import dataclasses
+import math
 from typing import Callable, Sequence
 
 import numpy as np
@@ -63,9 +75,15 @@ import numpy as np
 SOFTMAX_ALL_RENORM = 0
 SOFTMAX_TOPK = 1
 SIGMOID_TOPK_RENORM = 2
+SOFTMAX_ALL_NO_RENORM = 3
+
+ACT_SWIGLU = 0   # gated expert, three matrices (w_gate_up [2f, d], w_down [d, f])
+ACT_GELU = 1     # plain expert, two matrices (w_up [f, d], w_down [d, f])
 
 __all__ = [
-    "SOFTMAX_ALL_RENORM", "SOFTMAX_TOPK", "SIGMOID_TOPK_RENORM",
+    "SOFTMAX_ALL_RENORM", "SOFTMAX_TOPK", "SIGMOID_TOPK_RENORM", "SOFTMAX_ALL_NO_RENORM",
+    "ACT_SWIGLU", "ACT_GELU", "gelu", "gelu_expert", "expert_capacity", "dropped_slots",
+    "balance_loss", "router_z_loss", "logsumexp",
     "router_logits", "selection_key", "topk_select", "topk_gap", "softmax", "sigmoid",
     "gate_weights", "Routing", "route", "dispatch", "silu", "swiglu_expert", "moe_layer",
     "occupancy_closed_form", "occupancy_monte_carlo", "expert_params", "moe_layer_params",
@@ -131,6 +149,11 @@ def gate_weights(logits: np.ndarray, bias: np.ndarray | None, ids: np.ndarray, g
       expert, only the selected set is normalised.  With
       ``bias_select_only`` the score is the raw logit (bias steers selection
       only), else kappa.
+    * SOFTMAX_ALL_NO_RENORM -- [TOK] "How does MoE routing work": softmax over
+      all E, the selected experts' outputs combined with those probabilities
+      as they are (no renormalisation); with k = 1 this is [SEV] "Why top-1
+      routing cannot renormalise": the chosen expert scaled by the raw router
+      probability.
     """
     T, k = ids.shape
     key = selection_key(logits, bias)
@@ -146,6 +169,8 @@ def gate_weights(logits: np.ndarray, bias: np.ndarray | None, ids: np.ndarray, g
         score = logits if bias_select_only else key
         g = sigmoid(score)[rows, ids]
         return g / g.sum(axis=1, keepdims=True)
+    if gating == SOFTMAX_ALL_NO_RENORM:
+        return softmax(key, axis=1)[rows, ids]
     raise ValueError(f"unknown gating rule {gating}")
 
 
@@ -175,8 +200,21 @@ def route(x: np.ndarray, w_router: np.ndarray, bias: np.ndarray | None, k: int, 
 
 
 # ---------------------------------------------------------------- dispatch
-def dispatch(ids: np.ndarray, n_experts: int):
-    """Group the T*k (token, slot) assignments by expert, dropless.
+def expert_capacity(T: int, k: int, n_experts: int, capacity_factor: float) -> int:
+    """Most rows one expert takes in a batch: tokens per expert times the
+    capacity factor, rounded up ([TUR] "Capacity factor: when tokens don't
+    fit"; [SEV] counts routing slots, T*k/E, for top-k and rounds up).
+    Evaluated as ceil(((T*k)/E)*cf) in float64."""
+    return int(math.ceil(float(T * k) / float(n_experts) * float(capacity_factor)))
+
+
+def dropped_slots(counts: np.ndarray, capacity: int) -> int:
+    """Routing slots beyond the capacity, summed over experts ([SEV])."""
+    return int(sum(max(int(c) - capacity, 0) for c in counts))
+
+
+def dispatch(ids: np.ndarray, n_experts: int, capacity: int | None = None):
+    """Group the T*k (token, slot) assignments by expert.
 
     [TUR] "How data centres handle it": tokens are grouped by their assigned
     expert; [TUR] "Capacity factor": dropless means each expert gets exactly
@@ -184,27 +222,36 @@ def dispatch(ids: np.ndarray, n_experts: int):
     the assignments in order i = t*k + s gives, per expert in ascending
     order, its assignments in ascending token order:
 
-    counts[e]   number of rows of expert e          ([SEV] tokens per expert)
-    offsets     exclusive scan of counts, offsets[E] = T*k
+    counts[e]   number of assignments routed to expert e ([SEV] tokens per
+                expert: the router's demand, before any capacity cut)
+    offsets     exclusive scan of the rows each expert keeps, offsets[E] =
+                rows kept (T*k when dropless)
     perm[row]   = t*k + s, the assignment stored at that row
-    row_of[i]   = row of assignment i (inverse of perm)
+    row_of[i]   = row of assignment i (inverse of perm), -1 when dropped
+
+    With a ``capacity`` C an expert keeps its first C assignments in that
+    order and the rest skip it ([SEV]: "Tokens beyond that limit skip the
+    expert"); ``perm`` then has ``offsets[E]`` entries.
     """
     T, k = ids.shape
     flat = ids.reshape(-1)
     counts = np.zeros(n_experts, dtype=np.int64)
     for e in flat:
         counts[e] += 1
+    kept = counts if capacity is None else np.minimum(counts, capacity)
     offsets = np.zeros(n_experts + 1, dtype=np.int64)
     for e in range(n_experts):
-        offsets[e + 1] = offsets[e] + counts[e]
-    cursor = offsets[:-1].copy()
-    perm = np.empty(T * k, dtype=np.int64)
-    row_of = np.empty(T * k, dtype=np.int64)
+        offsets[e + 1] = offsets[e] + kept[e]
+    seen = np.zeros(n_experts, dtype=np.int64)
+    perm = np.empty(int(offsets[n_experts]), dtype=np.int64)
+    row_of = np.full(T * k, -1, dtype=np.int64)
     for i, e in enumerate(flat):
-        r = cursor[e]
-        cursor[e] += 1
-        perm[r] = i
-        row_of[i] = r
+        rank = seen[e]
+        seen[e] += 1
+        if rank < kept[e]:
+            r = offsets[e] + rank
+            perm[r] = i
+            row_of[i] = r
     return counts, offsets, perm, row_of
 
 
@@ -225,6 +272,22 @@ def swiglu_expert(xr: np.ndarray, w_gate: np.ndarray, w_up: np.ndarray, w_down: 
     return (silu(g) * u) @ w_down.T
 
 
+def gelu(z: np.ndarray) -> np.ndarray:
+    """GELU(z) = z * Phi(z) = z/2 * (1 + erf(z / sqrt 2)), the exact form
+    ([SEV]'s runnable build applies ``F.gelu`` between its two matrices)."""
+    from scipy.special import erf
+
+    z = np.asarray(z, dtype=np.float64)
+    return 0.5 * z * (1.0 + erf(z / math.sqrt(2.0)))
+
+
+def gelu_expert(xr: np.ndarray, w_up: np.ndarray, w_down: np.ndarray) -> np.ndarray:
+    """Two-matrix expert of [SEV]'s build: ``GELU(x W_up^T) W_down^T``.
+
+    xr [n, d], w_up [f, d], w_down [d, f]  ->  [n, d]."""
+    return gelu(xr @ w_up.T) @ w_down.T
+
+
 ExpertWeights = Callable[[int], tuple[np.ndarray, np.ndarray, np.ndarray]]
 
 
@@ -232,7 +295,8 @@ def moe_layer(x: np.ndarray, w_router: np.ndarray | None, bias: np.ndarray | Non
               expert_weights: ExpertWeights, n_experts: int,
               shared_weights: Sequence[tuple[np.ndarray, np.ndarray, np.ndarray]] = (),
               bias_select_only: int = 0, ids: np.ndarray | None = None,
-              decision_dtype=np.float32) -> tuple[np.ndarray, Routing | None, np.ndarray]:
+              decision_dtype=np.float32, act: int = ACT_SWIGLU,
+              capacity: int | None = None) -> tuple[np.ndarray, Routing | None, np.ndarray]:
     """Sparse MoE sublayer output for the tokens ``x`` [T, d].
 
     Router -> top-k -> per-expert loop -> weighted sum, as in [TUR]'s
@@ -241,7 +305,15 @@ def moe_layer(x: np.ndarray, w_router: np.ndarray | None, bias: np.ndarray | Non
     by that row's routing weight.  Shared experts ([TOK] "Shared experts";
     [TUR] "Shared expert and fine-grained experts") see every token, weight 1.
 
-    ``expert_weights(e)`` returns float64 ``(W_gate [f,d], W_up [f,d], W_down [d,f])``.
+    ``expert_weights(e)`` returns float64 ``(W_gate [f,d], W_up [f,d], W_down [d,f])``
+    for ``act = ACT_SWIGLU`` and ``(W_up [f,d], W_down [d,f])`` for ``ACT_GELU``
+    (the same for ``shared_weights``).
+
+    ``capacity``: when given, each expert processes only its first
+    ``capacity`` assignments in token order (:func:`dispatch`); a dropped
+    assignment adds nothing to its token's output and the other weights are
+    left as they are ([SEV]: a skipped token gets no expert update in that
+    layer; the residual connection that carries it lies outside this sublayer).
 
     Forced routing: when ``ids`` is given the selection is taken from it and
     only the gate weights and expert outputs are recomputed (``w_router``
@@ -258,16 +330,51 @@ def moe_layer(x: np.ndarray, w_router: np.ndarray | None, bias: np.ndarray | Non
         r = None
         ids_ = np.asarray(ids, dtype=np.int64)
         w = gate_weights(router_logits(x, w_router), bias, ids_, gating, bias_select_only)
+    keep = np.ones(ids_.shape, dtype=bool)
+    if capacity is not None:
+        _, _, _, row_of = dispatch(ids_, n_experts, capacity)
+        keep = (row_of >= 0).reshape(ids_.shape)
+
+    def ffn(xr, wts):
+        return swiglu_expert(xr, *wts) if act == ACT_SWIGLU else gelu_expert(xr, *wts)
+
     y = np.zeros_like(x)
     for e in range(n_experts):
-        rows, slots = np.nonzero(ids_ == e)
+        rows, slots = np.nonzero((ids_ == e) & keep)
         if rows.size == 0:
             continue
-        wg, wu, wd = expert_weights(e)
-        y[rows] += w[rows, slots][:, None] * swiglu_expert(x[rows], wg, wu, wd)
-    for wg, wu, wd in shared_weights:
-        y += swiglu_expert(x, wg, wu, wd)
+        y[rows] += w[rows, slots][:, None] * ffn(x[rows], expert_weights(e))
+    for wts in shared_weights:
+        y += ffn(x, wts)
     return y, r, w
+
+
+# ---------------------------------------------------------------- router penalties
+def logsumexp(v: np.ndarray, axis: int = -1) -> np.ndarray:
+    """log sum exp(v) = max + log sum exp(v - max)."""
+    m = np.max(v, axis=axis)
+    return m + np.log(np.sum(np.exp(v - np.expand_dims(m, axis)), axis=axis))
+
+
+def balance_loss(logits: np.ndarray, counts: np.ndarray) -> float:
+    """Load-balancing penalty of [SEV] (the top-1 routing paper's, extended to
+    top-k by counting routing slots), without its alpha:
+    ``N * sum_i f_i * P_i`` with f_i = share of the routed slots sent to
+    expert i and P_i = mean over tokens of the router's softmax probability
+    of expert i (softmax of the bias-free router logits).  Equals 1 for an
+    even split and N when every token goes to one expert with certainty."""
+    n = logits.shape[1]
+    c = np.asarray(counts, dtype=np.float64)
+    f = c / c.sum()
+    P = softmax(logits, axis=1).mean(axis=0)
+    return float(n * np.sum(f * P))
+
+
+def router_z_loss(logits: np.ndarray) -> float:
+    """Router z-loss ([TUR] "Router z-loss", [SEV]): the square of the
+    log-sum-exp of each token's router logits, averaged over tokens
+    (without the loss weight)."""
+    return float(np.mean(logsumexp(logits, axis=1) ** 2))
 
 
 # ---------------------------------------------------------------- occupancy

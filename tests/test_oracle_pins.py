@@ -367,3 +367,180 @@ def test_brute_force_exhaustive_tiny_routing():
             ids = oracle.topk_select(key, k)[0].tolist()
             ranked = sorted(range(4), key=lambda e: (-keyrow[e], e))
             assert ids == ranked[:k]
+
+
+# ------------------------------------------------------------------ routing without renormalisation
+def test_no_renorm_top1_weight_is_the_raw_router_probability():
+    """[SEV] "Why top-1 routing cannot renormalise": with k = 1 the chosen expert
+    is scaled by its raw router probability.  Reference: a pure-Python softmax
+    of each row, its largest entry.  Catches a renormalisation (weight 1) or a
+    softmax over the kept score only."""
+    rng = np.random.default_rng(41)
+    x = _rand(rng, 30, 10)
+    wr = _rand(rng, 6, 10, scale=0.8)
+    r = oracle.route(x, wr, None, 1, oracle.SOFTMAX_ALL_NO_RENORM, decision_dtype=None)
+    for t in range(30):
+        l = [_dot(x[t], wr[e]) for e in range(6)]
+        m = max(l)
+        z = math.fsum(math.exp(v - m) for v in l)
+        assert abs(r.w[t, 0] - max(math.exp(v - m) / z for v in l)) <= 1e-14
+        assert r.w[t, 0] < 1.0
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 6])
+def test_no_renorm_weights_are_the_unscaled_renorm_weights(k):
+    """[TOK] keeps the softmax probabilities as they are; [SEV] divides them by
+    their sum.  So the no-renormalisation weights, divided by their sum, are the
+    renormalised ones; their sum is at most 1 and exactly 1 at k = E."""
+    rng = np.random.default_rng(50 + k)
+    x = _rand(rng, 40, 8)
+    wr = _rand(rng, 6, 8)
+    bias = _rand(rng, 6, scale=0.5)
+    a = oracle.route(x, wr, bias, k, oracle.SOFTMAX_ALL_NO_RENORM)
+    b = oracle.route(x, wr, bias, k, oracle.SOFTMAX_ALL_RENORM)
+    assert np.array_equal(a.ids, b.ids)
+    s = a.w.sum(axis=1)
+    assert np.max(np.abs(a.w / s[:, None] - b.w)) <= 1e-14
+    assert np.all(s <= 1.0 + 1e-15)
+    if k == 6:
+        assert np.max(np.abs(s - 1.0)) <= 1e-14
+    else:
+        assert np.all(s < 1.0)
+
+
+# ------------------------------------------------------------------ capacity factor and token dropping
+def test_capacity_reproduces_the_page_cases():
+    """[SEV] capacity script on the page's printed tokens-per-expert line."""
+    g = json.loads((GOLDEN / "capacity_and_balance.json").read_text())
+    run = g["toy_run_counts"]
+    counts = np.array(run["tokens_per_expert"])
+    assert counts.sum() == run["tokens"] * run["top_k"]
+    for c in g["capacity_cases"]["cases"]:
+        cap = oracle.expert_capacity(run["tokens"], run["top_k"], run["n_experts"], c["factor"])
+        assert cap == c["capacity"]
+        assert oracle.dropped_slots(counts, cap) == c["dropped"]
+
+
+def test_capacity_rounds_up_not_down():
+    """ceil, not floor or round: 10 tokens x 1 / 3 experts x 1.0 = 3.33 -> 4."""
+    assert oracle.expert_capacity(10, 1, 3, 1.0) == 4
+    assert oracle.expert_capacity(9, 1, 3, 1.0) == 3
+    assert oracle.expert_capacity(8, 2, 8, 1.5) == 3
+
+
+@pytest.mark.parametrize("T,E,k,cap", [(40, 4, 2, 13), (57, 8, 3, 9), (25, 5, 5, 25), (30, 3, 1, 4), (12, 6, 2, 0)])
+def test_capacity_dispatch_keeps_the_first_arrivals(T, E, k, cap):
+    """Brute force: per expert, list its (token, slot) assignments in token
+    order and keep the first ``cap``.  Catches keeping the last arrivals,
+    ranking by slot instead of token, or offsets built from the raw counts."""
+    rng = np.random.default_rng(T * 100 + cap)
+    ids = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int64)
+    counts, offsets, perm, row_of = oracle.dispatch(ids, E, cap)
+    kept_rows = []
+    for e in range(E):
+        mine = [t * k + s for t in range(T) for s in range(k) if ids[t, s] == e]
+        assert counts[e] == len(mine)
+        kept_rows += mine[:cap]
+        for i in mine[cap:]:
+            assert row_of[i] == -1
+    assert list(perm) == kept_rows
+    assert offsets[-1] == len(kept_rows) == T * k - oracle.dropped_slots(counts, cap)
+    for r, i in enumerate(perm):
+        assert row_of[i] == r
+
+
+def test_capacity_layer_drops_expert_updates_and_keeps_other_weights():
+    """A dropped slot adds nothing; the token's other slots keep their weights
+    ([SEV]: a skipped token simply gets no expert update in that layer).
+    Reference: per-token loops over the kept slots."""
+    rng = np.random.default_rng(7)
+    x, wr, wgu, wd = _layer(rng, T=12, d=5, E=3, f=4)
+    k, cap = 2, 5
+    y, r, w = oracle.moe_layer(x, wr, None, k, oracle.SOFTMAX_TOPK, _experts(wgu, wd), 3, capacity=cap)
+    _, _, _, row_of = oracle.dispatch(r.ids, 3, cap)
+    f = wd.shape[2]
+    for t in range(12):
+        ref = [0.0] * 5
+        for s in range(k):
+            if row_of[t * k + s] < 0:
+                continue
+            e = int(r.ids[t, s])
+            o = _swiglu_loops(list(x[t]), wgu[e, :f].tolist(), wgu[e, f:].tolist(), wd[e].tolist())
+            ref = [a + w[t, s] * b for a, b in zip(ref, o)]
+        assert np.max(np.abs(y[t] - np.array(ref))) <= 1e-12
+    assert np.any(row_of < 0)  # the case does drop something
+
+
+def test_capacity_at_or_above_the_batch_is_dropless():
+    rng = np.random.default_rng(8)
+    x, wr, wgu, wd = _layer(rng, T=20, d=6, E=4, f=3)
+    a, *_ = oracle.moe_layer(x, wr, None, 2, oracle.SOFTMAX_TOPK, _experts(wgu, wd), 4)
+    b, *_ = oracle.moe_layer(x, wr, None, 2, oracle.SOFTMAX_TOPK, _experts(wgu, wd), 4, capacity=20)
+    assert np.array_equal(a, b)
+
+
+# ------------------------------------------------------------------ two-matrix GELU expert
+def test_gelu_special_values():
+    """GELU(z) = z * Phi(z): Phi(1) = 0.841344746068543 (normal table), GELU(0) = 0,
+    GELU(z) - GELU(-z) = z, GELU(z) -> z for large z and -> 0 for very negative z.
+    Catches the tanh approximation (GELU(1) = 0.841192) or a missing 1/2."""
+    g = oracle.gelu(np.array([1.0, 0.0, 2.5, -2.5, 30.0, -30.0]))
+    assert abs(g[0] - 0.8413447460685429) <= 1e-15
+    assert g[1] == 0.0
+    assert abs((g[2] - g[3]) - 2.5) <= 1e-15
+    assert g[4] == 30.0 and abs(g[5]) < 1e-150
+
+
+def test_gelu_single_expert_layer_is_the_pages_two_matrix_ffn():
+    """E = 1, k = 1: the layer is [SEV]'s Expert, down(GELU(up(x))), written here
+    with loops and math.erf."""
+    rng = np.random.default_rng(9)
+    T, d, f = 7, 5, 6
+    x = _rand(rng, T, d)
+    wup = _rand(rng, f, d, scale=0.6)
+    wdn = _rand(rng, d, f, scale=0.6)
+    y, _, _ = oracle.moe_layer(x, _rand(rng, 1, d), None, 1, oracle.SOFTMAX_TOPK, lambda e: (wup, wdn), 1,
+                               act=oracle.ACT_GELU)
+    for t in range(T):
+        h = []
+        for j in range(f):
+            z = _dot(x[t], wup[j])
+            h.append(0.5 * z * (1.0 + math.erf(z / math.sqrt(2.0))))
+        ref = [_dot(h, wdn[i]) for i in range(d)]
+        assert np.max(np.abs(y[t] - np.array(ref))) <= 1e-12
+
+
+# ------------------------------------------------------------------ router penalties
+def test_balance_loss_page_bounds():
+    """[SEV]: N * sum f_i P_i is 1 for an even split and N (8.0) when every
+    token goes to one expert with top-1 and certainty."""
+    g = json.loads((GOLDEN / "capacity_and_balance.json").read_text())["balance_loss_bounds"]
+    even = oracle.balance_loss(np.zeros((64, 8)), np.full(8, 16))
+    assert abs(even - g["even"]) <= 1e-15
+    peaked = np.full((64, 8), -1000.0)
+    peaked[:, 3] = 0.0
+    counts = np.zeros(8)
+    counts[3] = 64
+    assert abs(oracle.balance_loss(peaked, counts) - g["all_to_one_top1_n8"]) <= 1e-12
+
+
+def test_balance_loss_brute_force():
+    """Loops: f_i from the slot counts, P_i the mean of each token's softmax row."""
+    rng = np.random.default_rng(12)
+    l = _rand(rng, 20, 5, scale=2.0)
+    counts = np.array([7, 0, 13, 9, 11])
+    tot = 0.0
+    for i in range(5):
+        p_i = math.fsum(math.exp(l[t, i]) / math.fsum(math.exp(v) for v in l[t]) for t in range(20)) / 20
+        tot += counts[i] / counts.sum() * p_i
+    assert abs(oracle.balance_loss(l, counts) - 5 * tot) <= 1e-14
+
+
+def test_router_z_loss_closed_forms():
+    """Equal logits c: log-sum-exp = c + ln E, so the loss is (c + ln E)^2;
+    a shift by c does not leave it unchanged (unlike softmax)."""
+    assert abs(oracle.router_z_loss(np.zeros((9, 8))) - math.log(8) ** 2) <= 1e-14
+    assert abs(oracle.router_z_loss(np.full((3, 4), 2.0)) - (2.0 + math.log(4)) ** 2) <= 1e-13
+    l = np.array([[0.0, math.log(3.0)], [1.0, 1.0]])
+    ref = (math.log(1 + 3) ** 2 + (1 + math.log(2)) ** 2) / 2
+    assert abs(oracle.router_z_loss(l) - ref) <= 1e-14
