@@ -1,14 +1,17 @@
 /*
  * moe.h -- C ABI of the B200 (sm_100a) sparse Mixture-of-Experts layer forward.
  *
- * The layer (token-choice routing, dropless):
+ * The layer (token-choice routing, dropless unless a capacity is set):
  *   router logits   l = x W_r^T                                   [T, E]
  *   selection key   kappa = l + b        (b: optional per-expert bias)
  *   top-k           the k largest kappa per token, descending, ties -> lower index
- *   gate weights    one of three rules (moe_gating), fp32
- *   dispatch        rows grouped by expert (ascending), tokens ascending inside
+ *   gate weights    one of four rules (moe_gating), fp32
+ *   dispatch        rows grouped by expert (ascending), tokens ascending inside;
+ *                   with a capacity C each expert keeps its first C rows
  *   expert FFN      h = SiLU(x_e Wg^T) * (x_e Wu^T),  o = h Wd^T   (SwiGLU)
+ *                   or h = GELU(x_e Wu^T), o = h Wd^T               (moe_expert_act)
  *   combine         y[t] = sum_s w[t,s] o_{t,s} + sum_shared FFN_shared(x[t])
+ *                   (a dropped slot adds nothing)
  *
  * Sources (page title, section):
  *   "Mixture of Experts (MoE): routing, expert parallelism, and memory"
@@ -93,8 +96,23 @@ typedef enum {
   MOE_SOFTMAX_TOPK = 1,
   /* sigmoid score per expert, top-k, divide by the sum of the k
      ("...671 billion parameters uses only 37", sigmoid gating; DeepSeek-V3)  */
-  MOE_SIGMOID_TOPK_RENORM = 2
+  MOE_SIGMOID_TOPK_RENORM = 2,
+  /* softmax over all E kappas, the k kept probabilities used as they are
+     ("Mixture of Experts (MoE): routing...", "How does MoE routing work";
+     with k = 1 the raw router probability of top-1 routing, "Mixture of
+     Experts Explained...", "Why top-1 routing cannot renormalise")          */
+  MOE_SOFTMAX_ALL_NO_RENORM = 3
 } moe_gating;
+
+typedef enum {
+  /* gated expert, three matrices: h = SiLU(x Wg^T) * (x Wu^T), o = h Wd^T;
+     w_gate_up [E, 2f, d] (rows 0..f-1 Wg, f..2f-1 Wu)                       */
+  MOE_ACT_SWIGLU = 0,
+  /* plain expert, two matrices: h = GELU(x Wu^T) (exact erf form), o = h Wd^T;
+     the w_gate_up argument holds W_up [E, f, d]
+     ("Mixture of Experts Explained...", the runnable top-k MoE build)       */
+  MOE_ACT_GELU = 1
+} moe_expert_act;
 
 typedef struct {
   int64_t T;                /* tokens                                          */
@@ -107,8 +125,18 @@ typedef struct {
   int32_t dtype;            /* moe_dtype                                       */
   int32_t gating;           /* moe_gating                                      */
   int32_t bias_select_only; /* sigmoid rule: bias steers selection only        */
-  int32_t reserved;         /* must be 0                                       */
+  int32_t expert_act;       /* moe_expert_act (routed and shared experts)      */
   int64_t wait_limit_ns;    /* bound on any single device wait; 0 = 2 s        */
+  float capacity_factor;    /* 0: dropless.  > 0: every expert keeps only its
+                               first C = ceil(T*k/E * capacity_factor)
+                               assignments in token order; the rest skip it
+                               ("Mixture of Experts: why a model...",
+                               "Capacity factor: when tokens don't fit";
+                               "Mixture of Experts Explained...", expert
+                               capacity).  A dropped slot adds nothing to its
+                               token's output; the other slots keep their
+                               weights.                                        */
+  int32_t reserved;         /* must be 0                                       */
 } moe_config;
 
 /* Bytes of scratch every entry point below accepts for this config
@@ -119,6 +147,13 @@ size_t moe_workspace_bytes(const moe_config* cfg);
 /* Static, NUL-terminated description of a status code. */
 const char* moe_status_string(moe_status s);
 
+/* Rows each expert keeps: ceil(T*k/E * capacity_factor) evaluated in double
+   (capped at T, which no expert can exceed) when capacity_factor > 0, T*k
+   when it is 0 (dropless); -1 for an invalid config.  Host only.  With a
+   capacity C, the dropped slot count of a call is sum_e max(counts[e] - C, 0)
+   ("Mixture of Experts Explained...": dropped slots per capacity factor). */
+int64_t moe_expert_capacity(const moe_config* cfg);
+
 /* Router + top-k + gate weights, one fused pass.
    x [T, d] (dtype), w_router [E, d] (dtype), logit_bias [E] fp32 or NULL
    -> topk_ids [T, k] int32 (slots in descending kappa), topk_w [T, k] fp32. */
@@ -126,12 +161,37 @@ moe_status moe_router_topk(const moe_config* cfg, const void* x, const void* w_r
                            const float* logit_bias, int32_t* topk_ids, float* topk_w,
                            void* ws, size_t ws_bytes, moe_stream_t stream);
 
-/* Dropless dispatch: a stable counting sort of the T*k assignments by expert,
-   then the row gather.
+/* Router penalties of a batch, forward values only (training-side
+   quantities; the caller applies their loss weights):
+     out[0]  balance loss without alpha: E * sum_e f_e * P_e, with f_e =
+             counts[e] / sum(counts) the share of routed slots and P_e the mean
+             over tokens of the softmax probability of expert e
+             ("Mixture of Experts Explained...", the load-balancing loss of the
+             top-1 routing paper, counted over routing slots for top-k);
+     out[1]  router z-loss without its weight: the mean over tokens of
+             (log sum_e exp l[t,e])^2 ("Mixture of Experts: why a model...",
+             "Router z-loss").
+   Both use the bias-free router logits l = x W_r^T.  x [T, d], w_router
+   [E, d] (dtype), counts [E] int32 (routed slots per expert, as moe_permute
+   or moe_forward return them), out [2] fp32 device.  The logits are
+   recomputed on the CUDA cores; sums run in a fixed order (deterministic),
+   in fp32.  T = 0 writes zeros. */
+moe_status moe_router_aux_losses(const moe_config* cfg, const void* x, const void* w_router,
+                                 const int32_t* counts, float* out, void* ws, size_t ws_bytes,
+                                 moe_stream_t stream);
+
+/* Dispatch: a stable counting sort of the T*k assignments by expert, then
+   the row gather.
    topk_ids [T, k] int32, x [T, d]
-   -> counts [E], offsets [E+1] (exclusive scan, offsets[E] = T*k),
-      perm [T*k] (perm[row] = t*k + s), row_of [T*k] (inverse of perm),
-      x_perm [T*k, d] (x_perm[row] = x[perm[row] / k]).
+   -> counts [E] (assignments routed to each expert, before any capacity cut),
+      offsets [E+1] (exclusive scan of the rows each expert keeps:
+      min(counts[e], C) with a capacity C, counts[e] when dropless;
+      offsets[E] = rows kept, T*k when dropless),
+      perm [offsets[E]] (perm[row] = t*k + s),
+      row_of [T*k] (inverse of perm; -1 for a dropped assignment),
+      x_perm [offsets[E], d] (x_perm[row] = x[perm[row] / k]).
+   Rows inside an expert follow ascending token order, so with a capacity an
+   expert keeps its first C assignments in token order.
    Ids outside [0, E) are skipped and flag MOE_ERR_BAD_EXPERT_ID in the status
    word (read it with moe_device_status). */
 moe_status moe_permute(const moe_config* cfg, const int32_t* topk_ids, const void* x,

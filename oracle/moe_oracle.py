@@ -296,7 +296,8 @@ def moe_layer(x: np.ndarray, w_router: np.ndarray | None, bias: np.ndarray | Non
               shared_weights: Sequence[tuple[np.ndarray, np.ndarray, np.ndarray]] = (),
               bias_select_only: int = 0, ids: np.ndarray | None = None,
               decision_dtype=np.float32, act: int = ACT_SWIGLU,
-              capacity: int | None = None) -> tuple[np.ndarray, Routing | None, np.ndarray]:
+              capacity: int | None = None,
+              keep: np.ndarray | None = None) -> tuple[np.ndarray, Routing | None, np.ndarray]:
     """Sparse MoE sublayer output for the tokens ``x`` [T, d].
 
     Router -> top-k -> per-expert loop -> weighted sum, as in [TUR]'s
@@ -314,6 +315,8 @@ def moe_layer(x: np.ndarray, w_router: np.ndarray | None, bias: np.ndarray | Non
     assignment adds nothing to its token's output and the other weights are
     left as they are ([SEV]: a skipped token gets no expert update in that
     layer; the residual connection that carries it lies outside this sublayer).
+    ``keep`` ([T, k] bool) gives the kept slots directly, for evaluating a
+    subset of a batch whose drops were decided over the whole batch.
 
     Forced routing: when ``ids`` is given the selection is taken from it and
     only the gate weights and expert outputs are recomputed (``w_router``
@@ -330,10 +333,11 @@ def moe_layer(x: np.ndarray, w_router: np.ndarray | None, bias: np.ndarray | Non
         r = None
         ids_ = np.asarray(ids, dtype=np.int64)
         w = gate_weights(router_logits(x, w_router), bias, ids_, gating, bias_select_only)
-    keep = np.ones(ids_.shape, dtype=bool)
-    if capacity is not None:
-        _, _, _, row_of = dispatch(ids_, n_experts, capacity)
-        keep = (row_of >= 0).reshape(ids_.shape)
+    if keep is None:
+        keep = np.ones(ids_.shape, dtype=bool)
+        if capacity is not None:
+            _, _, _, row_of = dispatch(ids_, n_experts, capacity)
+            keep = (row_of >= 0).reshape(ids_.shape)
 
     def ffn(xr, wts):
         return swiglu_expert(xr, *wts) if act == ACT_SWIGLU else gelu_expert(xr, *wts)

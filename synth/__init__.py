@@ -49,6 +49,7 @@ STREAM_BIAS_PERM = 6
 SOFTMAX_ALL_RENORM = 0
 SOFTMAX_TOPK = 1
 SIGMOID_TOPK_RENORM = 2
+SOFTMAX_ALL_NO_RENORM = 3
 
 
 # --------------------------------------------------------------------------
@@ -181,6 +182,8 @@ class LayerConfig:
     zipf_s: float = 0.0    # 0: no routing bias; >0: Zipf(s) logit bias per expert
     bias_select_only: int = 0
     seed: int = 1000
+    act: int = 0           # 0: SwiGLU expert (gate+up rows), 1: GELU expert (up rows only)
+    capacity_factor: float = 0.0  # 0: dropless
 
     def replace(self, **kw) -> "LayerConfig":
         return dataclasses.replace(self, **kw)
@@ -211,16 +214,19 @@ DECODE_ZIPF_S = 1.2
 
 # element counts and standard deviations of every input tensor
 def tensor_specs(cfg: LayerConfig) -> dict[str, tuple[tuple[int, ...], int, float]]:
+    """``w_gate_up`` holds 2f rows per expert (gate, then up) for the SwiGLU
+    expert and f rows (up only) for the GELU expert."""
     d, E, f = cfg.d_model, cfg.n_experts, cfg.d_ff
+    m = 2 if cfg.act == 0 else 1
     specs = {
         "x": ((cfg.T, d), STREAM_X, 1.0),
         "w_router": ((E, d), STREAM_ROUTER, 1.0 / math.sqrt(d)),
-        "w_gate_up": ((E, 2 * f, d), STREAM_GATE_UP, 1.0 / math.sqrt(d)),
+        "w_gate_up": ((E, m * f, d), STREAM_GATE_UP, 1.0 / math.sqrt(d)),
         "w_down": ((E, d, f), STREAM_DOWN, 1.0 / math.sqrt(f)),
     }
     if cfg.n_shared:
         fs = cfg.d_ff_shared
-        specs["ws_gate_up"] = ((cfg.n_shared, 2 * fs, d), STREAM_SHARED_GATE_UP, 1.0 / math.sqrt(d))
+        specs["ws_gate_up"] = ((cfg.n_shared, m * fs, d), STREAM_SHARED_GATE_UP, 1.0 / math.sqrt(d))
         specs["ws_down"] = ((cfg.n_shared, d, fs), STREAM_SHARED_DOWN, 1.0 / math.sqrt(fs))
     return specs
 

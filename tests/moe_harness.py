@@ -31,7 +31,15 @@ def torch_dtype(cfg):
 def moe_cfg(cfg: synth.LayerConfig, T: int | None = None, wait_limit_ns: int = 0) -> moe.MoeConfig:
     return moe.make_config(cfg.T if T is None else T, cfg.d_model, cfg.n_experts, cfg.top_k, cfg.d_ff,
                            moe.MOE_BF16 if cfg.dtype == "bf16" else moe.MOE_F32, cfg.gating,
-                           cfg.n_shared, cfg.d_ff_shared, cfg.bias_select_only, wait_limit_ns)
+                           cfg.n_shared, cfg.d_ff_shared, cfg.bias_select_only, wait_limit_ns,
+                           expert_act=cfg.act, capacity_factor=cfg.capacity_factor)
+
+
+def capacity_of(cfg: synth.LayerConfig) -> int | None:
+    """The oracle's capacity for the workload (the factor as the float32 the ABI carries)."""
+    if cfg.capacity_factor == 0:
+        return None
+    return oracle.expert_capacity(cfg.T, cfg.top_k, cfg.n_experts, float(np.float32(cfg.capacity_factor)))
 
 
 def host_to_device(arr: np.ndarray, cfg, device="cuda") -> torch.Tensor:
@@ -95,29 +103,31 @@ class OracleWeights:
         if e in self._cache:
             return self._cache[e]
         f = self.cfg.d_ff
+        m = 2 if self.cfg.act == oracle.ACT_SWIGLU else 1
         if self.inp.on_host:
             d = self.cfg.d_model
-            gu = synth.host_tensor(self.cfg, "w_gate_up", e * 2 * f * d, 2 * f * d).reshape(2 * f, d)
+            gu = synth.host_tensor(self.cfg, "w_gate_up", e * m * f * d, m * f * d).reshape(m * f, d)
             wd = synth.host_tensor(self.cfg, "w_down", e * d * f, d * f).reshape(d, f)
         else:
             gu = device_to_host_f64(self.inp.dev["w_gate_up"][e])
             wd = device_to_host_f64(self.inp.dev["w_down"][e])
-        w = (gu[:f], gu[f:], wd)
+        w = (gu[:f], gu[f:], wd) if m == 2 else (gu, wd)
         if self.inp.on_host:  # full-size experts are refetched rather than held in host memory
             self._cache[e] = w
         return w
 
     def shared(self):
         out = []
+        m = 2 if self.cfg.act == oracle.ACT_SWIGLU else 1
         for s in range(self.cfg.n_shared):
             fs, d = self.cfg.d_ff_shared, self.cfg.d_model
             if self.inp.on_host:
-                gu = synth.host_tensor(self.cfg, "ws_gate_up", s * 2 * fs * d, 2 * fs * d).reshape(2 * fs, d)
+                gu = synth.host_tensor(self.cfg, "ws_gate_up", s * m * fs * d, m * fs * d).reshape(m * fs, d)
                 wd = synth.host_tensor(self.cfg, "ws_down", s * d * fs, d * fs).reshape(d, fs)
             else:
                 gu = device_to_host_f64(self.inp.dev["ws_gate_up"][s])
                 wd = device_to_host_f64(self.inp.dev["ws_down"][s])
-            out.append((gu[:fs], gu[fs:], wd))
+            out.append((gu[:fs], gu[fs:], wd) if m == 2 else (gu, wd))
         return out
 
     def w_router(self) -> np.ndarray:
@@ -192,16 +202,18 @@ def check_forward(inp: Inputs, out: dict, n_sample: int | None = None) -> dict:
     gpu_w = out["w"].cpu().numpy().astype(np.float64)
     r = oracle.route(x_all, wr, bias, k, cfg.gating, cfg.bias_select_only)
     stats = check_routing(cfg, gpu_ids, gpu_w, r, T)
-    counts, _offsets, _perm, _row_of = oracle.dispatch(gpu_ids, E)
+    cap = capacity_of(cfg)
+    counts, _offsets, _perm, row_of = oracle.dispatch(gpu_ids, E, cap)
     assert np.array_equal(out["counts"].cpu().numpy(), counts)
+    keep = (row_of >= 0).reshape(T, k)  # slots the capacity keeps, decided over the whole batch
     tokens = np.arange(T) if n_sample is None else sample_tokens(T, n_sample)
     y_ref, _, _ = oracle.moe_layer(x_all[tokens], wr, bias, k, cfg.gating, ow.routed, E,
                                    shared_weights=ow.shared(), bias_select_only=cfg.bias_select_only,
-                                   ids=gpu_ids[tokens])
+                                   ids=gpu_ids[tokens], act=cfg.act, keep=keep[tokens])
     y = device_to_host_f64(out["y"][torch.from_numpy(tokens).cuda()])
     err = rel_err(y, y_ref)
     assert err <= TOL[cfg.dtype], f"relative error {err:.3e} > {TOL[cfg.dtype]}"
     assert out["status"] == 0
     stats.update(rel_err=err, tokens_checked=len(tokens),
-                 experts_touched=int(np.sum(counts > 0)))
+                 experts_touched=int(np.sum(counts > 0)), dropped=int(np.sum(~keep)))
     return stats

@@ -85,5 +85,20 @@ def test_host_checks_reject_before_launch(L):
 
 
 def test_config_struct_layout():
-    assert ctypes.sizeof(moe.MoeConfig) == 56
+    assert ctypes.sizeof(moe.MoeConfig) == 64
+    assert moe.MoeConfig.expert_act.offset == 44
     assert moe.MoeConfig.wait_limit_ns.offset == 48
+    assert moe.MoeConfig.capacity_factor.offset == 56
+
+
+def test_expert_capacity_host_arithmetic(L):
+    """ceil(T*k/E * factor) on the host, T*k when dropless, capped at T."""
+    assert moe.moe_expert_capacity(_cfg(T=512, top_k=2, n_experts=8, capacity_factor=1.25)) == 160
+    assert moe.moe_expert_capacity(_cfg(T=512, top_k=2, n_experts=8, capacity_factor=1.0)) == 128
+    assert moe.moe_expert_capacity(_cfg(T=10, top_k=1, n_experts=3, d_ff=8, capacity_factor=1.0)) == 4
+    assert moe.moe_expert_capacity(_cfg(T=64, top_k=2)) == 128
+    assert moe.moe_expert_capacity(_cfg(T=64, top_k=2, capacity_factor=100.0)) == 64
+    assert moe.moe_expert_capacity(_cfg(capacity_factor=-1.0)) == -1
+    assert moe.moe_expert_capacity(_cfg(capacity_factor=float("nan"))) == -1
+    assert moe.moe_expert_capacity(_cfg(expert_act=2)) == -1
+    assert moe.moe_expert_capacity(_cfg(gating=4)) == -1

@@ -32,6 +32,31 @@ SMALL = {
     "k_equals_E": synth.LayerConfig("k_equals_E", 64, 256, 4, 4, 256, "bf16", synth.SOFTMAX_ALL_RENORM, seed=16),
     "single_expert": synth.LayerConfig("single_expert", 200, 256, 1, 1, 384, "bf16", synth.SOFTMAX_TOPK, seed=17),
     "one_token": synth.LayerConfig("one_token", 1, 512, 8, 2, 512, "bf16", synth.SOFTMAX_TOPK, seed=18),
+    # softmax weights kept without renormalisation; k = 1 is the raw top-1 probability
+    "norenorm_top1": synth.LayerConfig("norenorm_top1", 300, 256, 8, 1, 256, "bf16", synth.SOFTMAX_ALL_NO_RENORM,
+                                       seed=22),
+    "norenorm_f32_k3": synth.LayerConfig("norenorm_f32_k3", 150, 136, 6, 3, 72, "f32", synth.SOFTMAX_ALL_NO_RENORM,
+                                         zipf_s=0.7, seed=23),
+    "norenorm_tc_router": synth.LayerConfig("norenorm_tc_router", 270, 256, 64, 2, 128, "bf16",
+                                            synth.SOFTMAX_ALL_NO_RENORM, seed=24),
+    # capacity factor with token dropping (Zipf-skewed routing so that some experts overflow)
+    "capacity_1_0": synth.LayerConfig("capacity_1_0", 333, 256, 8, 2, 384, "bf16", synth.SOFTMAX_TOPK,
+                                      zipf_s=1.2, capacity_factor=1.0, seed=25),
+    "capacity_f32_0_5": synth.LayerConfig("capacity_f32_0_5", 200, 128, 4, 2, 96, "f32", synth.SOFTMAX_ALL_RENORM,
+                                          zipf_s=1.0, capacity_factor=0.5, seed=26),
+    "capacity_shared": synth.LayerConfig("capacity_shared", 257, 512, 64, 8, 256, "bf16", synth.SIGMOID_TOPK_RENORM,
+                                         n_shared=1, d_ff_shared=384, zipf_s=1.0, bias_select_only=1,
+                                         capacity_factor=1.25, seed=27),
+    # two-matrix GELU experts
+    "gelu_bf16": synth.LayerConfig("gelu_bf16", 300, 256, 8, 2, 320, "bf16", synth.SOFTMAX_ALL_RENORM, act=1,
+                                   seed=28),
+    "gelu_decode_bf16": synth.LayerConfig("gelu_decode_bf16", 20, 512, 16, 2, 384, "bf16", synth.SOFTMAX_TOPK,
+                                          act=1, seed=29),
+    "gelu_f32_shared": synth.LayerConfig("gelu_f32_shared", 140, 128, 6, 2, 200, "f32", synth.SOFTMAX_ALL_RENORM,
+                                         n_shared=1, d_ff_shared=136, act=1, seed=30),
+    "gelu_capacity_shared": synth.LayerConfig("gelu_capacity_shared", 200, 256, 16, 4, 192, "bf16",
+                                              synth.SOFTMAX_ALL_NO_RENORM, n_shared=1, d_ff_shared=256, act=1,
+                                              zipf_s=1.0, capacity_factor=0.8, seed=31),
 }
 
 
@@ -95,7 +120,7 @@ def test_zero_tokens_is_a_no_op():
 
 # ------------------------------------------------------------------ single entry points
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("gating", [0, 1, 2])
+@pytest.mark.parametrize("gating", [0, 1, 2, 3])
 @pytest.mark.parametrize("E,k", [(8, 2), (64, 6), (256, 8)])
 def test_router_topk(dtype, gating, E, k):
     cfg = synth.LayerConfig("r", 333, 264, E, k, 8, dtype, gating, zipf_s=1.1, bias_select_only=1, seed=E + k)
@@ -114,7 +139,8 @@ def test_router_topk(dtype, gating, E, k):
 
 @pytest.mark.parametrize("T,E,k", [(1, 1, 1), (1000, 8, 2), (4099, 256, 8), (2048, 1024, 16), (333, 5, 5)])
 @pytest.mark.parametrize("skew", ["uniform", "one_expert", "half_empty"])
-def test_permute_bit_exact(T, E, k, skew):
+@pytest.mark.parametrize("cf", [0.0, 1.0, 0.3])
+def test_permute_bit_exact(T, E, k, skew, cf):
     rng = np.random.default_rng(T + E + k)
     if skew == "uniform":
         keys = rng.random((T, E))
@@ -127,8 +153,10 @@ def test_permute_bit_exact(T, E, k, skew):
     ids = np.argsort(-keys, axis=1, kind="stable")[:, :k].astype(np.int32)
     d = 136
     x = rng.standard_normal((T, d)).astype(np.float32)
-    cfg = synth.LayerConfig("p", T, d, E, k, 8, "f32", 0)
+    cfg = synth.LayerConfig("p", T, d, E, k, 8, "f32", 0, capacity_factor=cf)
     c = H.moe_cfg(cfg)
+    cap = H.capacity_of(cfg)
+    assert moe.moe_expert_capacity(c) == (T * k if cap is None else min(cap, T))
     ws = torch.zeros(moe.moe_workspace_bytes(c), dtype=torch.uint8, device="cuda")
     dids = torch.from_numpy(ids).cuda()
     dx = torch.from_numpy(x).cuda()
@@ -139,12 +167,13 @@ def test_permute_bit_exact(T, E, k, skew):
     x_perm = torch.empty(T * k, d, dtype=torch.float32, device="cuda")
     moe.moe_permute(c, dids, dx, counts, offsets, perm, row_of, x_perm, ws)
     assert moe.moe_device_status(ws) == 0
-    rc, ro, rp, rr = oracle.dispatch(ids.astype(np.int64), E)
+    rc, ro, rp, rr = oracle.dispatch(ids.astype(np.int64), E, cap)
+    n_kept = int(ro[-1])
     assert np.array_equal(counts.cpu().numpy(), rc)
     assert np.array_equal(offsets.cpu().numpy(), ro)
-    assert np.array_equal(perm.cpu().numpy(), rp)
+    assert np.array_equal(perm.cpu().numpy()[:n_kept], rp)
     assert np.array_equal(row_of.cpu().numpy(), rr)
-    assert np.array_equal(x_perm.cpu().numpy(), x[rp // k])
+    assert np.array_equal(x_perm.cpu().numpy()[:n_kept], x[rp // k])
 
 
 def test_permute_flags_out_of_range_ids():
@@ -177,8 +206,10 @@ def _ragged_offsets(sizes):
     ([5, 0, 140], 264, 200),                     # partial n-tiles in both GEMMs
     ([1000], 512, 1024),                          # one big group
     ([3] * 40, 128, 136),                         # many tiny groups
-    ([70, 0, 1, 64, 65], 4096, 640),              # decode kernel: 2-chunk groups, split-K GEMM-1
-    ([1, 1], 4096, 14336),                        # decode kernel: one token per expert, split-K GEMM-2
+    ([70, 0, 1, 64, 65], 4096, 640),              # decode schedule: 2-chunk groups, split reductions
+    ([1, 1], 4096, 14336),                        # decode schedule: one token per expert
+    ([3, 0, 40, 1], 1024, 1536),                  # decode schedule: units cut across several CTAs
+    ([2100, 17, 0, 256, 257], 256, 192),          # 256-token chunks, a 9-chunk group, N = 16 remainders
 ])
 def test_grouped_ffn_against_dense_experts(dtype, sizes, d, f):
     rng = np.random.default_rng(sum(sizes) + d + f)
@@ -210,6 +241,41 @@ def test_grouped_ffn_against_dense_experts(dtype, sizes, d, f):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("sizes,d,f", [
+    ([0, 1, 127, 129, 300, 0, 256], 256, 384),   # large-batch schedule
+    ([3, 0, 40, 1], 1024, 1536),                  # decode schedule, units cut across CTAs
+    ([600, 17], 264, 200),                        # partial weight blocks, N = 32 remainder
+])
+def test_grouped_ffn_gelu_against_dense_experts(dtype, sizes, d, f):
+    """Two-matrix experts: y = GELU(a Wu^T) Wd^T per group."""
+    rng = np.random.default_rng(sum(sizes) + d + f + 1)
+    G = len(sizes)
+    rows = int(sum(sizes))
+    offs = _ragged_offsets(sizes)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    a = torch.from_numpy(rng.standard_normal((rows, d)).astype(np.float32)).to(tdt).cuda()
+    wu = torch.from_numpy((rng.standard_normal((G, f, d)) / np.sqrt(d)).astype(np.float32)).to(tdt).cuda()
+    wd = torch.from_numpy((rng.standard_normal((G, d, f)) / np.sqrt(f)).astype(np.float32)).to(tdt).cuda()
+    y = torch.full((rows, d), float("nan"), dtype=tdt, device="cuda")
+    cfg = synth.LayerConfig("g", rows, d, G, 1, f, dtype, 0, act=1)
+    c = H.moe_cfg(cfg)
+    ws = torch.zeros(moe.moe_workspace_bytes(c), dtype=torch.uint8, device="cuda")
+    moe.moe_grouped_ffn(c, a, torch.from_numpy(offs).cuda(), wu, wd, y, ws)
+    assert moe.moe_device_status(ws) == 0
+    A = H.device_to_host_f64(a)
+    WU = H.device_to_host_f64(wu)
+    WD = H.device_to_host_f64(wd)
+    ref = np.zeros((rows, d))
+    for g in range(G):
+        r0, r1 = offs[g], offs[g + 1]
+        if r1 > r0:
+            ref[r0:r1] = oracle.gelu_expert(A[r0:r1], WU[g], WD[g])
+    got = H.device_to_host_f64(y)
+    assert not np.any(np.isnan(got))
+    assert H.rel_err(got, ref) <= H.TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("shared", [False, True])
 def test_combine(dtype, shared):
     rng = np.random.default_rng(3)
@@ -228,3 +294,37 @@ def test_combine(dtype, shared):
     if shared:
         ref += H.device_to_host_f64(ys)
     assert H.rel_err(H.device_to_host_f64(y), ref) <= (1e-6 if dtype == "f32" else 8e-3)
+
+
+# ------------------------------------------------------------------ router penalties
+@pytest.mark.parametrize("dtype,E,k,d,T", [("bf16", 8, 2, 512, 700), ("bf16", 256, 8, 1024, 333),
+                                           ("f32", 12, 3, 264, 190), ("bf16", 64, 1, 256, 1)])
+def test_router_aux_losses(dtype, E, k, d, T):
+    """Balance loss (without alpha) and z-loss from the bias-free logits, against
+    the oracle on the same stored inputs and the GPU's own routed-slot counts.
+    Relative tolerance 1e-4: fp32 logits and fp32 sums in a fixed order."""
+    cfg = synth.LayerConfig("aux", T, d, E, k, 8, dtype, synth.SOFTMAX_TOPK, zipf_s=1.1, seed=E + T)
+    inp = H.make_inputs(cfg)
+    c = H.moe_cfg(cfg)
+    ws = torch.zeros(moe.moe_workspace_bytes(c), dtype=torch.uint8, device="cuda")
+    ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    moe.moe_router_topk(c, inp.dev["x"], inp.dev["w_router"], inp.dev["bias"], ids, w, ws)
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    row_of = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    x_perm = torch.empty(T * k, d, dtype=H.torch_dtype(cfg), device="cuda")
+    moe.moe_permute(c, ids, inp.dev["x"], counts, offsets, perm, row_of, x_perm, ws)
+    out = torch.full((4,), float("nan"), dtype=torch.float32, device="cuda")
+    moe.moe_router_aux_losses(c, inp.dev["x"], inp.dev["w_router"], counts, out, ws)
+    assert moe.moe_device_status(ws) == 0
+    x = synth.host_tensor(cfg, "x").reshape(T, d)
+    wr = synth.host_tensor(cfg, "w_router").reshape(E, d)
+    logits = oracle.router_logits(x, wr)
+    cnt = counts.cpu().numpy()
+    ref = (oracle.balance_loss(logits, cnt), oracle.router_z_loss(logits))
+    got = out.cpu().numpy()
+    assert abs(got[0] - ref[0]) <= 1e-4 * abs(ref[0]), (got, ref)
+    assert abs(got[1] - ref[1]) <= 1e-4 * abs(ref[1]), (got, ref)
+    assert np.isnan(got[2]) and np.isnan(got[3])  # nothing written past out[1]

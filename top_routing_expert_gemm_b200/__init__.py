@@ -13,8 +13,9 @@ import pathlib
 __all__ = [
     "MoeError", "MoeConfig", "lib", "make_config", "moe_workspace_bytes", "moe_status_string",
     "moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_forward", "moe_device_status",
-    "moe_permute_noalloc",
+    "moe_permute_noalloc", "moe_expert_capacity", "moe_router_aux_losses",
     "MOE_F32", "MOE_BF16", "MOE_SOFTMAX_ALL_RENORM", "MOE_SOFTMAX_TOPK", "MOE_SIGMOID_TOPK_RENORM",
+    "MOE_SOFTMAX_ALL_NO_RENORM", "MOE_ACT_SWIGLU", "MOE_ACT_GELU",
     "EXPORTED_SYMBOLS", "LIB_PATH",
 ]
 
@@ -24,11 +25,13 @@ MOE_OK = 0
 MOE_ERR_TIMEOUT = 5
 MOE_ERR_BAD_EXPERT_ID = 6
 MOE_F32, MOE_BF16 = 0, 1
-MOE_SOFTMAX_ALL_RENORM, MOE_SOFTMAX_TOPK, MOE_SIGMOID_TOPK_RENORM = 0, 1, 2
+MOE_SOFTMAX_ALL_RENORM, MOE_SOFTMAX_TOPK, MOE_SIGMOID_TOPK_RENORM, MOE_SOFTMAX_ALL_NO_RENORM = 0, 1, 2, 3
+MOE_ACT_SWIGLU, MOE_ACT_GELU = 0, 1
 
 EXPORTED_SYMBOLS = (
     "moe_workspace_bytes", "moe_status_string", "moe_router_topk", "moe_permute", "moe_grouped_ffn",
-    "moe_combine", "moe_forward", "moe_device_status", "moe_permute_noalloc",
+    "moe_combine", "moe_forward", "moe_device_status", "moe_permute_noalloc", "moe_expert_capacity",
+    "moe_router_aux_losses",
 )
 
 
@@ -50,8 +53,10 @@ class MoeConfig(ctypes.Structure):
         ("dtype", ctypes.c_int32),
         ("gating", ctypes.c_int32),
         ("bias_select_only", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("expert_act", ctypes.c_int32),
         ("wait_limit_ns", ctypes.c_int64),
+        ("capacity_factor", ctypes.c_float),
+        ("reserved", ctypes.c_int32),
     ]
 
 
@@ -78,17 +83,21 @@ def lib() -> ctypes.CDLL:
         L.moe_forward.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_device_status.argtypes = [vp, sz, vp]
         L.moe_permute_noalloc.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.moe_expert_capacity.argtypes = [cfgp]
+        L.moe_router_aux_losses.argtypes = [cfgp, vp, vp, vp, vp, vp, sz, vp]
         for name in EXPORTED_SYMBOLS[2:]:
             getattr(L, name).restype = i32
+        L.moe_expert_capacity.restype = ctypes.c_int64
         _lib = L
     return _lib
 
 
 def make_config(T: int, d_model: int, n_experts: int, top_k: int, d_ff: int, dtype: int, gating: int,
                 n_shared: int = 0, d_ff_shared: int = 0, bias_select_only: int = 0,
-                wait_limit_ns: int = 0) -> MoeConfig:
+                wait_limit_ns: int = 0, expert_act: int = MOE_ACT_SWIGLU,
+                capacity_factor: float = 0.0) -> MoeConfig:
     return MoeConfig(T, d_model, n_experts, top_k, d_ff, n_shared, d_ff_shared, dtype, gating,
-                     bias_select_only, 0, wait_limit_ns)
+                     bias_select_only, expert_act, wait_limit_ns, capacity_factor, 0)
 
 
 def _p(v) -> int | None:
@@ -122,10 +131,22 @@ def moe_workspace_bytes(cfg: MoeConfig) -> int:
     return int(lib().moe_workspace_bytes(ctypes.byref(cfg)))
 
 
+def moe_expert_capacity(cfg: MoeConfig) -> int:
+    """Rows each expert keeps (T*k when dropless); -1 for an invalid config."""
+    return int(lib().moe_expert_capacity(ctypes.byref(cfg)))
+
+
 def moe_router_topk(cfg, x, w_router, logit_bias, topk_ids, topk_w, ws, ws_bytes=None, stream=None) -> None:
     nb = ws_bytes if ws_bytes is not None else ws.numel() * ws.element_size()
     _check(lib().moe_router_topk(ctypes.byref(cfg), _p(x), _p(w_router), _p(logit_bias), _p(topk_ids),
                                  _p(topk_w), _p(ws), nb, _stream(stream)), "moe_router_topk")
+
+
+def moe_router_aux_losses(cfg, x, w_router, counts, out, ws, ws_bytes=None, stream=None) -> None:
+    """out[0] = balance loss (without alpha), out[1] = router z-loss (without its weight)."""
+    nb = ws_bytes if ws_bytes is not None else ws.numel() * ws.element_size()
+    _check(lib().moe_router_aux_losses(ctypes.byref(cfg), _p(x), _p(w_router), _p(counts), _p(out), _p(ws), nb,
+                                       _stream(stream)), "moe_router_aux_losses")
 
 
 def moe_permute(cfg, topk_ids, x, counts, offsets, perm, row_of, x_perm, ws, ws_bytes=None, stream=None) -> None:

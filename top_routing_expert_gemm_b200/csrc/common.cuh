@@ -50,6 +50,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 // SiLU(z) = z / (1 + e^-z), written with the CUDA math library's expf
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
+// GELU(z) = z * Phi(z) = z/2 * (1 + erf(z / sqrt 2)), with the CUDA math library's erff
+__device__ __forceinline__ float gelu_f(float z) { return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f)); }
+
+// expert activations (moe_expert_act) and the epilogue of the second GEMM
+constexpr int kEpiSwiGLU = 0, kEpiGELU = 1, kEpiNone = 2;
 
 __device__ __forceinline__ void set_status(int* status, int code) {
   if (status) atomicMax(status, code);

@@ -1,12 +1,14 @@
-// fp32 grouped SwiGLU experts on CUDA cores (no TF32: the fp32 layer keeps a
-// 24-bit mantissa end to end).  Same grouping contract as the tensor-core
-// path: rows [offsets[g], offsets[g+1]) of A use weight group g.
+// fp32 grouped experts on CUDA cores (no TF32: the fp32 layer keeps a 24-bit
+// mantissa end to end).  Same grouping contract as the tensor-core path: rows
+// [offsets[g], offsets[g+1]) of A use weight group g.
 //
 //   GEMM-1 + SwiGLU : h = SiLU(A Wg^T) * (A Wu^T)     (gate rows 0..f-1, up rows f..2f-1)
+//   GEMM-1 + GELU   : h = GELU(A Wu^T)                (two-matrix expert)
 //   GEMM-2          : y = h Wd^T
 //
-// Expert FFN reading: "Mixture of Experts Explained: Routers, Active
-// Parameters and VRAM" (a gated feed-forward block with three matrices).
+// Expert FFN: "Mixture of Experts Explained: Routers, Active Parameters and
+// VRAM" (a gated feed-forward block with three matrices; the runnable build's
+// two-matrix expert with GELU between them).
 // 64x64 output tiles, K in steps of 16 through shared memory, 4x4 outputs per
 // thread.  The grid covers an upper bound of the (group, m-tile) pairs; each
 // block finds its pair from the device offsets, so no host sync is needed.
@@ -44,12 +46,13 @@ __device__ bool find_group_tile(const int32_t* offsets, int G, int64_t rows, int
   return false;
 }
 
-template <bool SWIGLU>
+template <int EPI>
 __global__ void __launch_bounds__(kThreads) grouped_gemm_f32_kernel(const float* __restrict__ A, int64_t rows,
                                                                     const int32_t* __restrict__ offsets, int G,
                                                                     const float* __restrict__ W,
                                                                     int64_t w_group_rows, int up_off, int K,
                                                                     int N, float* __restrict__ out) {
+  constexpr bool SWIGLU = EPI == kEpiSwiGLU;
   __shared__ float As[BK][BM + 4];
   __shared__ float Bs[SWIGLU ? 2 : 1][BK][BN + 4];
   __shared__ int s_g;
@@ -117,7 +120,9 @@ __global__ void __launch_bounds__(kThreads) grouped_gemm_f32_kernel(const float*
     for (int j = 0; j < 4; ++j) {
       const int c = n0 + tx * 4 + j;
       if (c >= N) continue;
-      out[(row0 + r) * N + c] = SWIGLU ? silu_f(acc0[i][j]) * acc1[i][j] : acc0[i][j];
+      out[(row0 + r) * N + c] = EPI == kEpiSwiGLU ? silu_f(acc0[i][j]) * acc1[i][j]
+                                : EPI == kEpiGELU  ? gelu_f(acc0[i][j])
+                                                   : acc0[i][j];
     }
   }
 }
@@ -128,11 +133,16 @@ cudaError_t launch_grouped_ffn_f32_simt(const GroupedFfnArgs& a, cudaStream_t st
   if (a.rows == 0) return cudaSuccess;
   const int64_t mt_bound = (a.rows + BM - 1) / BM + (a.offsets ? a.G : 0);
   const dim3 grid1((unsigned)mt_bound, (unsigned)((a.f + BN - 1) / BN));
-  grouped_gemm_f32_kernel<true><<<grid1, kThreads, 0, stream>>>(
-      static_cast<const float*>(a.a), a.rows, a.offsets, a.G, static_cast<const float*>(a.w_gate_up),
-      2 * (int64_t)a.f, a.f, a.d, a.f, static_cast<float*>(a.h));
+  if (a.act == kEpiGELU)
+    grouped_gemm_f32_kernel<kEpiGELU><<<grid1, kThreads, 0, stream>>>(
+        static_cast<const float*>(a.a), a.rows, a.offsets, a.G, static_cast<const float*>(a.w_gate_up),
+        (int64_t)a.f, 0, a.d, a.f, static_cast<float*>(a.h));
+  else
+    grouped_gemm_f32_kernel<kEpiSwiGLU><<<grid1, kThreads, 0, stream>>>(
+        static_cast<const float*>(a.a), a.rows, a.offsets, a.G, static_cast<const float*>(a.w_gate_up),
+        2 * (int64_t)a.f, a.f, a.d, a.f, static_cast<float*>(a.h));
   const dim3 grid2((unsigned)mt_bound, (unsigned)((a.d + BN - 1) / BN));
-  grouped_gemm_f32_kernel<false><<<grid2, kThreads, 0, stream>>>(
+  grouped_gemm_f32_kernel<kEpiNone><<<grid2, kThreads, 0, stream>>>(
       static_cast<const float*>(a.h), a.rows, a.offsets, a.G, static_cast<const float*>(a.w_down), a.d, 0, a.f,
       a.d, static_cast<float*>(a.y));
   return cudaGetLastError();

@@ -1,0 +1,579 @@
+// Grouped expert GEMMs on the sm_100a tensor cores with the operands swapped:
+// an expert's weight rows are the MMA's M operand (128 rows) and its tokens
+// the N operand, so the MMA width follows the expert's token count (rounded up
+// to 16) instead of a fixed 128-row token tile.  An expert with 270 tokens
+// costs 256 + 16 MMA columns rather than three 128-row tiles, and an expert
+// with 3 tokens costs 16.
+//
+// "Mixture of Experts: why a model with 671 billion parameters uses only 37",
+// "How data centres handle it" (tokens grouped by expert, all expert
+// multiplies in one launch over a stacked weight matrix) and "Capacity factor:
+// when tokens don't fit" (dropless: every expert gets exactly its rows, no
+// padding to a fixed size); "Mixture of experts: how MoE works and what it
+// costs", "What mixture of experts costs in compute" (decode per-expert
+// batches are small and memory bound).  Expert FFN: "Mixture of Experts
+// Explained: Routers, Active Parameters and VRAM" (a gated feed-forward block
+// with three matrices), read as SwiGLU.
+//
+//   GEMM-1 (SwiGLU): h^T[f-block, tokens] = [Wg; Wu][64+64 rows] x_perm^T;
+//     accumulator rows 0..63 are gate rows, 64..127 the matching up rows; the
+//     epilogue pairs them through shared memory and writes h[tokens, f].
+//   GEMM-1 (GELU, the two-matrix expert): h^T = GELU(Wu[128 rows] x_perm^T).
+//   GEMM-2 (plain):  y^T[d-block, tokens] = Wd[128 rows] h^T.
+//
+// A unit is (expert, weight-row block j, token chunk of up to BN tokens).
+// Inside an expert the units run over blocks of 8 chunks, then j, then the
+// chunk: units running together share weight blocks and token chunks through
+// L2 even for an expert with thousands of tokens.
+//
+// Two schedules (template STREAMK):
+//   * large batches (BN = 256): unit u runs on CTA u mod gridDim (persistent
+//     CTAs, every unit whole);
+//   * decode (BN = 64, STREAMK): the reduction steps of all units, laid end to
+//     end, are cut into one equal contiguous range per CTA, so every CTA
+//     streams the same number of weight bytes whatever the routing.  A unit
+//     cut between CTAs is finished by the last contributor to arrive: each
+//     writes its fp32 partial tile (at most two per CTA: its first and last
+//     unit), adds its step count to the unit's counter, and the one that
+//     completes the count sums the partials in CTA order -- a fixed order, so
+//     results are deterministic -- and runs the epilogue.  Nothing waits on
+//     another CTA.
+//
+// Persistent, warp-specialised CTA (192 threads): warp 0 TMA producer, warp 1
+// TMEM allocator and single-thread tcgen05.mma issuer, warps 2-5 epilogue;
+// two accumulators of BN columns so the epilogue of one unit overlaps the
+// main loop of the next.  Every wait is bounded; on expiry the CTA raises an
+// abort flag and the device status word, drains its own copies and MMAs,
+// frees its tensor memory and returns.
+#include <algorithm>
+#include <cmath>
+
+#include "kernels.cuh"
+#include "tc_primitives.cuh"
+
+namespace moe {
+namespace tc {
+namespace {
+
+constexpr int S_BK = 64;
+constexpr int S_BM = 128;                   // weight rows per MMA (SwiGLU: 64 gate + 64 up)
+constexpr int S_THREADS = 192;
+constexpr int S_XG = 17;                    // pitch (floats) of a gate/up exchange row: 16 tokens + 1
+constexpr int S_HP = 136;                   // pitch (bf16) of a staged output row: 128 columns + 8
+// epilogue staging: exchange [2][64][S_XG] fp32, then outputs [32][S_HP] bf16
+constexpr int S_STAGE_BYTES = 2 * 64 * S_XG * 4 + 32 * S_HP * 2;
+constexpr int S_CB = 8;                     // token chunks per block in the unit order
+constexpr int S_A_BYTES = S_BM * S_BK * 2;  // 16 KiB
+constexpr int kDevInternal = 7;             // status word: internal size check failed
+
+template <int BN>
+struct Shape {
+  static constexpr int STAGES = BN <= 64 ? 8 : 4;
+  static constexpr int B_BYTES = BN * S_BK * 2;
+  static constexpr int TMEM_COLS = 2 * BN;
+};
+
+struct SwapParams {
+  const int32_t* offsets;  // [G+1] token-row offsets, or null: one group of `rows`
+  int G;
+  int64_t rows;            // token rows of B and of the output
+  int K;                   // reduction length
+  int n_out;               // output columns (f or d)
+  int J;                   // weight-row blocks per group
+  int64_t a_group_rows;    // weight rows per group (2f or d)
+  int up_off;              // f (SwiGLU)
+  __nv_bfloat16* out;      // [rows, n_out]
+  int64_t ldo;
+  float* partial;          // STREAMK: [2 * gridDim.x][128][BN] fp32 partial tiles
+  int* counters;           // STREAMK: one per unit; zero on entry, zero on exit
+  int64_t counter_cap;     // units the counters (and the schedule) allow
+  int* status;
+  uint64_t wait_limit_ns;
+};
+
+template <int BN>
+size_t swap_smem_bytes(int G) {
+  return 1024 + (size_t)Shape<BN>::STAGES * (S_A_BYTES + Shape<BN>::B_BYTES) + S_STAGE_BYTES + 256 +
+         2 * sizeof(int) * (size_t)(G + 1);
+}
+
+// Named barrier of the four epilogue warps (barrier 1, 128 threads).
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Same barrier, returning whether any of the 128 threads passed true: the
+// epilogue warps use it to take their loop-exit decision together.
+__device__ __forceinline__ bool epi_bar_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pin, pout;\n\t"
+      "setp.ne.u32 pin, %1, 0;\n\t"
+      "bar.red.or.pred pout, 1, 128, pin;\n\t"
+      "selp.u32 %0, 1, 0, pout;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+struct Unit {
+  int g, j, chunk;
+  int n_valid;  // tokens of this chunk (1..BN)
+  int nmma;     // MMA N: n_valid rounded up to 16
+};
+
+// unit -> (group, weight block, token chunk)
+__device__ __forceinline__ Unit decode_unit(int64_t u, int J, const int* cum, const int* off, int G, int bn) {
+  int lo = 0, hi = G;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if ((int64_t)cum[mid] * J <= u) lo = mid;
+    else hi = mid;
+  }
+  Unit r;
+  r.g = lo;
+  const int nch = cum[lo + 1] - cum[lo];
+  const int64_t local = u - (int64_t)cum[lo] * J;
+  const int cb = (int)(local / ((int64_t)S_CB * J));
+  const int64_t rest = local - (int64_t)cb * S_CB * J;
+  const int nb = min(S_CB, nch - cb * S_CB);  // chunks in this block
+  r.j = (int)(rest / nb);
+  r.chunk = cb * S_CB + (int)(rest % nb);
+  r.n_valid = min(bn, off[lo + 1] - off[lo] - r.chunk * bn);
+  r.nmma = (r.n_valid + 15) & ~15;
+  return r;
+}
+
+// First reduction step of CTA c's range when `total` steps are cut into `parts`.
+__device__ __forceinline__ int64_t range_start(int64_t c, int64_t total, int64_t parts) { return c * total / parts; }
+// The CTA whose range holds step i.
+__device__ __forceinline__ int64_t range_owner(int64_t i, int64_t total, int64_t parts) {
+  return ((i + 1) * parts - 1) / total;
+}
+
+// Calls f(unit, kb0, kb1, first) for this CTA's segments in order, until f returns false.
+template <bool STREAMK, typename F>
+__device__ __forceinline__ void for_each_segment(int64_t n_units, int kb_count, F&& f) {
+  if (STREAMK) {
+    const int64_t total = n_units * kb_count, parts = gridDim.x;
+    const int64_t begin = range_start(blockIdx.x, total, parts), end = range_start(blockIdx.x + 1, total, parts);
+    for (int64_t pos = begin; pos < end;) {
+      const int64_t u = pos / kb_count;
+      const int kb0 = (int)(pos - u * kb_count);
+      const int kb1 = (end - pos < (int64_t)(kb_count - kb0)) ? kb0 + (int)(end - pos) : kb_count;
+      const bool first = pos == begin;
+      pos += kb1 - kb0;
+      if (!f(u, kb0, kb1, first)) return;
+    }
+  } else {
+    for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x)
+      if (!f(u, 0, kb_count, true)) return;
+  }
+}
+
+template <int EPI, int BN, bool STREAMK>
+__global__ void __launch_bounds__(S_THREADS, 1)
+    grouped_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX64,
+                             const __grid_constant__ CUtensorMap tmX16, const SwapParams p) {
+  constexpr int STAGES = Shape<BN>::STAGES;
+  constexpr int B_BYTES = Shape<BN>::B_BYTES;
+  constexpr bool SWIGLU = EPI == kEpiSwiGLU;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * S_A_BYTES;
+  float* xg = reinterpret_cast<float*>(sB + STAGES * B_BYTES);  // [64][S_XG] gate values, tokens 16..31
+  float* xu = xg + 64 * S_XG;                                    // [64][S_XG] up values, tokens 0..15
+  __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(xu + 64 * S_XG);  // [32][S_HP] staged outputs
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES + S_STAGE_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = bars + 2 * STAGES + 2;
+  uint64_t* drain = bars + 2 * STAGES + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* reducer_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  int* fill_par = reinterpret_cast<int*>(tmem_slot + 3);  // [STAGES]
+  int* s_off = fill_par + STAGES;                          // [G+1]
+  int* s_cum = s_off + (p.G + 1);                          // [G+1] cumulative token chunks
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int G = p.G;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+      fill_par[s] = -1;
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&tfull[a]), 1);
+      mbar_init(smem_u32(&tempty[a]), 128);
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX64);
+    tma_prefetch_desc(&tmX16);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), Shape<BN>::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (p.offsets) {
+    for (int g = threadIdx.x; g <= G; g += S_THREADS) s_off[g] = p.offsets[g];
+  } else if (threadIdx.x == 0) {
+    s_off[0] = 0;
+    s_off[1] = (int)p.rows;
+  }
+  __syncthreads();
+  if (warp == 0) {  // cumulative BN-token chunks per group
+    int carry = 0;
+    if (lane == 0) s_cum[0] = 0;
+    for (int base = 0; base < G; base += 32) {
+      const int g = base + lane;
+      int v = 0;
+      if (g < G) v = max(0, (s_off[g + 1] - s_off[g] + BN - 1) / BN);
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += u;
+      }
+      if (g < G) s_cum[g + 1] = carry + v;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem_base = *tmem_slot;
+  const int kb_count = (p.K + S_BK - 1) / S_BK;
+  int64_t n_units = (int64_t)s_cum[G] * p.J;
+  if (n_units > p.counter_cap) {  // the host sized the schedule for fewer units: do nothing
+    if (threadIdx.x == 0) set_status(p.status, kDevInternal);
+    n_units = 0;
+  }
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      for_each_segment<STREAMK>(n_units, kb_count, [&](int64_t u, int kb0, int kb1, bool) {
+        const Unit un = decode_unit(u, p.J, s_cum, s_off, G, BN);
+        const int w_row = (int)((int64_t)un.g * p.a_group_rows + (int64_t)un.j * (SWIGLU ? S_BM / 2 : S_BM));
+        const int x_row = s_off[un.g] + un.chunk * BN;
+        const uint32_t tx = S_A_BYTES + (uint32_t)un.nmma * S_BK * 2;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait_bounded(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, p.wait_limit_ns, p.status))
+            return false;
+          const uint32_t fb = smem_u32(&full[stage]);
+          mbar_expect_tx(fb, tx);
+          fill_par[stage] = (int)phase;
+          const uint32_t a_dst = smem_u32(sA + stage * S_A_BYTES);
+          if (SWIGLU) {  // 64 gate rows, then the 64 matching up rows
+            tma_load_2d(a_dst, &tmW, fb, kb * S_BK, w_row);
+            tma_load_2d(a_dst + S_A_BYTES / 2, &tmW, fb, kb * S_BK, w_row + p.up_off);
+          } else {
+            tma_load_2d(a_dst, &tmW, fb, kb * S_BK, w_row);
+          }
+          const uint32_t b_dst = smem_u32(sB + stage * B_BYTES);
+          int b = 0;
+          for (; b + 64 <= un.nmma; b += 64) tma_load_2d(b_dst + b * S_BK * 2, &tmX64, fb, kb * S_BK, x_row + b);
+          for (; b < un.nmma; b += 16) tma_load_2d(b_dst + b * S_BK * 2, &tmX16, fb, kb * S_BK, x_row + b);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        return true;
+      });
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for_each_segment<STREAMK>(n_units, kb_count, [&](int64_t u, int kb0, int kb1, bool) {
+        const Unit un = decode_unit(u, p.J, s_cum, s_off, G, BN);
+        const uint32_t idesc = idesc_bf16_f32(S_BM, un.nmma);
+        if (!mbar_wait_bounded(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, p.wait_limit_ns, p.status))
+          return false;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait_bounded(smem_u32(&full[stage]), phase, abort_flag, p.wait_limit_ns, p.status)) return false;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * S_A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < S_BK / 16; ++kk)
+            mma_bf16(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32), idesc,
+                     (kb != kb0 || kk != 0) ? 1u : 0u);
+          mma_commit(smem_u32(&empty[stage]));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        mma_commit(smem_u32(&tfull[acc]));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+        return true;
+      });
+    }
+  } else {
+    // -------------------------------------------------- epilogue (warps 2..5)
+    const int q = warp & 3;
+    const int r = q * 32 + lane;  // accumulator row = weight row inside the block
+    const bool leader = (warp == 2 && lane == 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+
+    // Final epilogue of 32 token columns [32 cc, 32 cc + 32) of a unit.  The
+    // outputs are staged token-major in shared memory and leave in coalesced
+    // 16-byte stores.  SwiGLU: a gate row and its up row sit in different
+    // warps, so gate rows finish tokens 0..15 and up rows tokens 16..31, each
+    // taking the other half's partner values through shared memory.
+    auto finish = [&](const Unit& un, const float (&v)[32], int cc) {
+      const int nv = min(32, un.n_valid - 32 * cc);
+      const int64_t row0 = (int64_t)s_off[un.g] + (int64_t)un.chunk * BN + 32 * cc;
+      int ncols, col0;
+      if (SWIGLU) {
+        const int f = r & 63;
+        if (r < 64) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) xg[f * S_XG + i] = v[16 + i];
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) xu[f * S_XG + i] = v[i];
+        }
+        epi_bar();
+        if (r < 64) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) hs[i * S_HP + f] = __float2bfloat16_rn(silu_f(v[i]) * xu[f * S_XG + i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            hs[(16 + i) * S_HP + f] = __float2bfloat16_rn(silu_f(xg[f * S_XG + i]) * v[16 + i]);
+        }
+        ncols = 64;
+        col0 = un.j * 64;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) hs[i * S_HP + r] = __float2bfloat16_rn(EPI == kEpiGELU ? gelu_f(v[i]) : v[i]);
+        ncols = S_BM;
+        col0 = un.j * S_BM;
+      }
+      epi_bar();
+      const int segs = ncols / 8;  // 16-byte segments per token row
+      for (int c = r; c < 32 * segs; c += 128) {
+        const int tok = c / segs, sg = c % segs;
+        const int col = col0 + sg * 8;
+        const int64_t row = row0 + tok;
+        if (tok < nv && row < p.rows) {
+          const __nv_bfloat16* src = hs + tok * S_HP + sg * 8;
+          __nv_bfloat16* dst = p.out + row * p.ldo + col;
+          if (col + 8 <= p.n_out) {
+            *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+          } else {
+            for (int e = 0; e < 8; ++e)
+              if (col + e < p.n_out) dst[e] = src[e];
+          }
+        }
+      }
+      epi_bar();  // the staging buffers are free again
+    };
+
+    for_each_segment<STREAMK>(n_units, kb_count, [&](int64_t u, int kb0, int kb1, bool first) {
+      const Unit un = decode_unit(u, p.J, s_cum, s_off, G, BN);
+      const bool got = mbar_wait_bounded(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.wait_limit_ns, p.status);
+      if (epi_bar_any(!got || *abort_flag)) return false;  // every epilogue warp leaves together
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      const int nc32 = (un.nmma + 31) / 32;
+      float v[32];
+      if (kb0 == 0 && kb1 == kb_count) {  // the whole unit is here
+        for (int cc = 0; cc < nc32; ++cc) {
+          uint32_t raw[32];
+          tmem_ld32(tb + 32 * cc, raw);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
+          finish(un, v, cc);
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&tempty[acc]));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+        return true;
+      }
+      // part of a unit: publish this CTA's partial; the contributor that
+      // completes the unit's step count sums them all
+      const int64_t slot = 2 * (int64_t)blockIdx.x + (first ? 0 : 1);
+      float* prow = p.partial + (slot * S_BM + r) * BN;
+      for (int cc = 0; cc < nc32; ++cc) {
+        uint32_t raw[32];
+        tmem_ld32(tb + 32 * cc, raw);
+        tmem_ld_wait();
+        float4* dst = reinterpret_cast<float4*>(prow + 32 * cc);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (32 * cc + 4 * i < un.nmma)
+            dst[i] = make_float4(__uint_as_float(raw[4 * i]), __uint_as_float(raw[4 * i + 1]),
+                                 __uint_as_float(raw[4 * i + 2]), __uint_as_float(raw[4 * i + 3]));
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&tempty[acc]));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+      __threadfence();
+      epi_bar();
+      if (leader) *reducer_flag = (atomicAdd(&p.counters[u], kb1 - kb0) + (kb1 - kb0) == kb_count);
+      epi_bar();
+      // (the leader rewrites the flag only after the next segment's
+      // epi_bar_any, which every reader has passed by then)
+      if (!*reducer_flag) return true;
+      __threadfence();
+      const int64_t total = n_units * kb_count, parts = gridDim.x;
+      const int64_t c0 = range_owner(u * kb_count, total, parts);
+      const int64_t c1 = range_owner(u * kb_count + kb_count - 1, total, parts);
+      for (int cc = 0; cc < nc32; ++cc) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        for (int64_t c = c0; c <= c1; ++c) {  // contributors in CTA order = K order
+          const int64_t cs = range_start(c, total, parts);
+          if (range_start(c + 1, total, parts) == cs) continue;  // empty range: no partial
+          const int64_t s2 = 2 * c + (cs / kb_count == u ? 0 : 1);
+          const float4* src = reinterpret_cast<const float4*>(p.partial + (s2 * S_BM + r) * BN + 32 * cc);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (32 * cc + 4 * i < un.nmma) {
+              const float4 w4 = __ldcg(src + i);
+              v[4 * i] += w4.x;
+              v[4 * i + 1] += w4.y;
+              v[4 * i + 2] += w4.z;
+              v[4 * i + 3] += w4.w;
+            }
+          }
+        }
+        finish(un, v, cc);
+      }
+      if (leader) p.counters[u] = 0;  // ready for the next launch
+      return true;
+    });
+  }
+
+  if (warp == 0 && lane == 0 && !*abort_flag) {
+    // every stage filled has been released by its MMAs (their completion
+    // arrivals target this CTA's barriers, which must outlive them)
+    for (int s = 0; s < STAGES; ++s)
+      if (fill_par[s] >= 0) drain_wait(smem_u32(&empty[s]), (uint32_t)fill_par[s]);
+  }
+  __syncthreads();
+  if (*abort_flag) {
+    if (warp == 0 && lane == 0) {
+      for (int s = 0; s < STAGES; ++s)
+        if (fill_par[s] >= 0) drain_wait(smem_u32(&full[s]), (uint32_t)fill_par[s]);
+    }
+    if (warp == 1 && lane == 0) {
+      mma_commit(smem_u32(drain));
+      drain_wait(smem_u32(drain), 0);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Shape<BN>::TMEM_COLS);
+  }
+}
+
+template <int EPI, int BN, bool STREAMK>
+cudaError_t launch_swap(const CUtensorMap& tw, const CUtensorMap& tx64, const CUtensorMap& tx16,
+                        const SwapParams& p, int grid, cudaStream_t stream) {
+  auto kernel = grouped_gemm_swap_kernel<EPI, BN, STREAMK>;
+  const size_t smem = swap_smem_bytes<BN>(p.G);
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  if (STREAMK) {  // the counters must read zero on entry (a launch that timed out may leave some set)
+    e = cudaMemsetAsync(p.counters, 0, sizeof(int) * (size_t)p.counter_cap, stream);
+    if (e != cudaSuccess) return e;
+  }
+  kernel<<<(unsigned)grid, S_THREADS, smem, stream>>>(tw, tx64, tx16, p);
+  return cudaGetLastError();
+}
+
+// Units of one GEMM, bounded from the row count (the chunking is per group).
+int64_t unit_bound(int64_t rows, int G, int bn, int J) { return ((rows + bn - 1) / bn + G) * (int64_t)J; }
+
+// Both GEMMs of the expert FFN with one schedule.
+template <int BN, bool STREAMK>
+cudaError_t run_swap(const GroupedFfnArgs& a, cudaStream_t stream) {
+  const int G = a.offsets ? a.G : 1;
+  const uint64_t lim = a.wait_limit_ns ? a.wait_limit_ns : 2000000000ull;
+  const int sms = device_sm_count();
+  const bool gelu = a.act == kEpiGELU;
+  const int J1 = gelu ? (a.f + 127) / 128 : (a.f + 63) / 64, J2 = (a.d + 127) / 128;
+  const int64_t cap1 = unit_bound(a.rows, G, BN, J1), cap2 = unit_bound(a.rows, G, BN, J2);
+  if (STREAMK && (cap1 > a.counter_cap || cap2 > a.counter_cap)) return cudaErrorInvalidValue;
+  auto grid_for = [&](int64_t cap) -> int {
+    int64_t g = STREAMK ? std::min(sms, kDecodeMaxCtas) : std::min<int64_t>(sms, cap);
+    return (int)std::max<int64_t>(g, 1);
+  };
+  // GEMM-1: SwiGLU weight blocks of 64 gate + 64 up rows, or GELU blocks of
+  // 128 up rows; tokens of x_perm
+  const int64_t w1_rows = (gelu ? 1 : 2) * (int64_t)a.f;
+  CUtensorMap w1, x1a, x1b;
+  if (!make_map(&w1, a.w_gate_up, (uint64_t)a.G * w1_rows, a.d, gelu ? S_BM : 64) ||
+      !make_map(&x1a, a.a, a.rows, a.d, 64) || !make_map(&x1b, a.a, a.rows, a.d, 16))
+    return cudaErrorInvalidValue;
+  SwapParams p1{a.offsets, G, a.rows, a.d, a.f, J1, w1_rows, a.f, static_cast<__nv_bfloat16*>(a.h), a.f,
+                a.partial, a.counters, STREAMK ? a.counter_cap : cap1, a.status, lim};
+  cudaError_t e = gelu ? launch_swap<kEpiGELU, BN, STREAMK>(w1, x1a, x1b, p1, grid_for(cap1), stream)
+                       : launch_swap<kEpiSwiGLU, BN, STREAMK>(w1, x1a, x1b, p1, grid_for(cap1), stream);
+  if (e != cudaSuccess) return e;
+  // GEMM-2: weight blocks of 128 down rows, tokens of h
+  CUtensorMap w2, x2a, x2b;
+  if (!make_map(&w2, a.w_down, (uint64_t)a.G * a.d, a.f, S_BM) || !make_map(&x2a, a.h, a.rows, a.f, 64) ||
+      !make_map(&x2b, a.h, a.rows, a.f, 16))
+    return cudaErrorInvalidValue;
+  SwapParams p2{a.offsets, G, a.rows, a.f, a.d, J2, (int64_t)a.d, 0, static_cast<__nv_bfloat16*>(a.y), a.d,
+                a.partial, a.counters, STREAMK ? a.counter_cap : cap2, a.status, lim};
+  return launch_swap<kEpiNone, BN, STREAMK>(w2, x2a, x2b, p2, grid_for(cap2), stream);
+}
+
+}  // namespace
+}  // namespace tc
+
+bool use_decode_ffn(int64_t rows, int G, bool grouped) {
+  double touched = grouped ? G * (1.0 - std::pow(1.0 - 1.0 / G, (double)rows)) : 1.0;
+  if (touched < 1.0) touched = 1.0;
+  return (double)rows / touched <= kDecodeTokens;
+}
+
+// Partial tiles of the decode schedule: two [128][kDecodeTokens] fp32 tiles per CTA.
+int64_t decode_partial_slots() { return 2 * (int64_t)kDecodeMaxCtas; }
+
+// Units (expert, weight block, token chunk) of either GEMM of the decode schedule.
+int64_t decode_counter_cap(int64_t rows, int G, int d, int f) {
+  return tc::unit_bound(rows, G, kDecodeTokens, std::max((f + 63) / 64, (d + 127) / 128));
+}
+
+cudaError_t launch_grouped_ffn_bf16_decode(const GroupedFfnArgs& a, cudaStream_t stream) {
+  if (a.rows == 0) return cudaSuccess;
+  if (a.partial == nullptr || a.counters == nullptr || a.partial_slots < decode_partial_slots())
+    return cudaErrorInvalidValue;
+  return tc::run_swap<kDecodeTokens, true>(a, stream);
+}
+
+cudaError_t launch_grouped_ffn_bf16_swap(const GroupedFfnArgs& a, cudaStream_t stream) {
+  if (a.rows == 0) return cudaSuccess;
+  return tc::run_swap<256, false>(a, stream);
+}
+
+}  // namespace moe

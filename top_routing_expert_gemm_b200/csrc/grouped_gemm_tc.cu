@@ -11,6 +11,7 @@
 //     the matching N/2 up columns (the B tile is the gate rows followed by the
 //     up rows), so the SwiGLU is applied in the epilogue straight out of
 //     tensor memory and only h (bf16) reaches HBM.
+//   GEMM-1 (MODE_GELU, the two-matrix expert): h[rows, f] = GELU(A Wu^T).
 //   GEMM-2 (MODE_PLAIN):  y[rows, d] = h Wd^T.
 //   Router (MODE_ROUTER): logits = x W_r^T with N = E rounded up to 16; the
 //     epilogue keeps the top k per row and writes ids and gate weights.
@@ -76,7 +77,7 @@ constexpr int BN_MMA = 256;
 constexpr int A_BYTES = BM * BK * 2;       // 16 KiB
 constexpr int B_BYTES = BN_MMA * BK * 2;   // 32 KiB
 constexpr int TMEM_COLS = 2 * BN_MMA;      // two accumulators
-constexpr int MODE_SWIGLU = 0, MODE_PLAIN = 1, MODE_ROUTER = 2;
+constexpr int MODE_SWIGLU = 0, MODE_PLAIN = 1, MODE_ROUTER = 2, MODE_GELU = 3;
 
 struct Params {
   const int32_t* offsets;  // [G+1] device, or null: one group of `rows` rows
@@ -308,6 +309,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 h0 = silu_f(h0) * __uint_as_float(u[2 * j]);
                 h1 = silu_f(h1) * __uint_as_float(u[2 * j + 1]);
               }
+              if (MODE == MODE_GELU) {
+                h0 = gelu_f(h0);
+                h1 = gelu_f(h1);
+              }
               pk[j] = pack_bf16x2(h0, h1);
             }
             if (col_base + c + 32 <= col_lim) {
@@ -347,7 +352,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
         float z = 0.f;
-        if (p.gating == 0) {  // softmax over all E: needs the full denominator
+        if (p.gating == 0 || p.gating == 3) {  // softmax over all E: needs the full denominator
 #pragma unroll 1
           for (int c = 0; c < p.n_mma; c += 32) {
             uint32_t v[32];
@@ -365,7 +370,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int s = 0; s < KMAX; ++s) {
             float wv = 0.f;
             if (s < p.k) {
-              if (p.gating == 0) wv = expf(tk.key[s] - mx) / z;
+              if (p.gating == 0 || p.gating == 3) wv = expf(tk.key[s] - mx) / z;
               else if (p.gating == 1) wv = expf(tk.key[s] - tk.key[0]);
               else wv = 1.0f / (1.0f + expf(-(p.bias_select_only ? tk.val[s] : tk.key[s])));
             }
@@ -376,7 +381,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int s = 0; s < KMAX; ++s) {
             if (s < p.k) {
               p.ids[grow * p.k + s] = tk.idx[s];
-              p.wts[grow * p.k + s] = wsel[s] / den;
+              p.wts[grow * p.k + s] = p.gating == 3 ? wsel[s] : wsel[s] / den;  // rule 3: not renormalised
             }
           }
         }
@@ -439,15 +444,24 @@ cudaError_t launch_grouped_ffn_bf16_tc(const GroupedFfnArgs& a, cudaStream_t str
   const int G = a.offsets ? a.G : 1;
   const int64_t mt_bound = (a.rows + BM - 1) / BM + (a.offsets ? a.G : 0);
   const uint64_t lim = a.wait_limit_ns ? a.wait_limit_ns : 2000000000ull;
-  // GEMM-1 + SwiGLU: tile = 128 rows x (128 gate + 128 up) columns.  Narrower
-  // or non-power-of-two MMA widths measured slower on the layer shapes here.
   const int n1 = BN_MMA;
   CUtensorMap mA1, mB1;
-  if (!make_map(&mA1, a.a, a.rows, a.d, BM) || !make_map(&mB1, a.w_gate_up, (uint64_t)a.G * 2 * a.f, a.d, n1 / 2))
-    return cudaErrorInvalidValue;
-  Params p1{a.offsets, G, a.rows, a.d, a.f, (a.f + n1 / 2 - 1) / (n1 / 2), 2 * (int64_t)a.f, a.f, a.h, a.f,
-            a.status, lim, n1};
-  cudaError_t e = launch_mode<MODE_SWIGLU, 1>(mA1, mB1, p1, mt_bound * p1.nt, stream);
+  cudaError_t e;
+  if (a.act == kEpiGELU) {
+    // GEMM-1 + GELU: tile = 128 rows x 256 up columns
+    if (!make_map(&mA1, a.a, a.rows, a.d, BM) || !make_map(&mB1, a.w_gate_up, (uint64_t)a.G * a.f, a.d, n1))
+      return cudaErrorInvalidValue;
+    Params p1{a.offsets, G, a.rows, a.d, a.f, (a.f + n1 - 1) / n1, (int64_t)a.f, 0, a.h, a.f, a.status, lim, n1};
+    e = launch_mode<MODE_GELU, 1>(mA1, mB1, p1, mt_bound * p1.nt, stream);
+  } else {
+    // GEMM-1 + SwiGLU: tile = 128 rows x (128 gate + 128 up) columns.  Narrower
+    // or non-power-of-two MMA widths measured slower on the layer shapes here.
+    if (!make_map(&mA1, a.a, a.rows, a.d, BM) || !make_map(&mB1, a.w_gate_up, (uint64_t)a.G * 2 * a.f, a.d, n1 / 2))
+      return cudaErrorInvalidValue;
+    Params p1{a.offsets, G, a.rows, a.d, a.f, (a.f + n1 / 2 - 1) / (n1 / 2), 2 * (int64_t)a.f, a.f, a.h, a.f,
+              a.status, lim, n1};
+    e = launch_mode<MODE_SWIGLU, 1>(mA1, mB1, p1, mt_bound * p1.nt, stream);
+  }
   if (e != cudaSuccess) return e;
   // GEMM-2: tile = 128 rows x 256 output columns
   const int n2 = BN_MMA;

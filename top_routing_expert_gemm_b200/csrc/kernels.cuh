@@ -20,10 +20,17 @@ struct RouterArgs {
   bool bf16;
   int* status;
   uint64_t wait_limit_ns;
+  // router penalties only: per-block sums [blocks][E + 1] (softmax probabilities
+  // of the bias-free logits per expert, then squared log-sum-exp), or null
+  float* aux_part;
 };
+constexpr int kAuxMaxBlocks = 2048;  // router blocks of a penalty pass, at most
 cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t stream);       // picks one of:
 cudaError_t launch_router_topk_simt(const RouterArgs& a, cudaStream_t stream);  // CUDA cores, any dtype
 cudaError_t launch_router_topk_tc(const RouterArgs& a, cudaStream_t stream);    // tcgen05, bf16, E <= 256
+// The CUDA-core router with the penalty sums (a.aux_part set), then the
+// reduction into out[0] = balance loss, out[1] = z-loss.
+cudaError_t launch_router_aux_losses(const RouterArgs& a, const int32_t* counts, float* out, cudaStream_t stream);
 
 // ---- dispatch (permute.cu)
 struct PermuteArgs {
@@ -39,6 +46,7 @@ struct PermuteArgs {
   int k, d, E;
   int elem_bytes;
   int* status;
+  int64_t capacity;       // rows each expert keeps (n_assign or more: dropless)
 };
 int permute_n_chunks(int64_t n_assign);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream);
@@ -49,26 +57,31 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream);
 struct GroupedFfnArgs {
   const void* a;          // [rows, d]
   const int32_t* offsets; // [G+1] or null
-  const void* w_gate_up;  // [G, 2f, d]
+  const void* w_gate_up;  // [G, 2f, d] (SwiGLU) or [G, f, d] (GELU: up rows only)
   const void* w_down;     // [G, d, f]
   void* h;                // [rows, f] scratch
   void* y;                // [rows, d]
   int64_t rows;           // rows of a / h / y (T*k, or T for a shared expert)
   int G, d, f;
+  int act;                // kEpiSwiGLU or kEpiGELU
   int* status;
   uint64_t wait_limit_ns;
-  // decode kernel only: split-K partial tiles and per-tile arrival counters
+  // decode kernel only: fp32 partial tiles of units cut between CTAs, and
+  // one arrival counter per unit
   float* partial;
   int64_t partial_slots;
   int* counters;
   int64_t counter_cap;
 };
-cudaError_t launch_grouped_ffn_bf16_tc(const GroupedFfnArgs& a, cudaStream_t stream);      // tcgen05, large batch
-cudaError_t launch_grouped_ffn_bf16_decode(const GroupedFfnArgs& a, cudaStream_t stream);  // tcgen05, swap-AB
+constexpr int kDecodeMaxCtas = 160;  // CTAs of one decode-schedule launch, at most
+constexpr int kDecodeTokens = 64;    // most tokens per unit of the decode schedule
+cudaError_t launch_grouped_ffn_bf16_tc(const GroupedFfnArgs& a, cudaStream_t stream);      // tcgen05, token rows as M
+cudaError_t launch_grouped_ffn_bf16_swap(const GroupedFfnArgs& a, cudaStream_t stream);    // tcgen05, weight rows as M
+cudaError_t launch_grouped_ffn_bf16_decode(const GroupedFfnArgs& a, cudaStream_t stream);  // the same, split reductions
 cudaError_t launch_grouped_ffn_f32_simt(const GroupedFfnArgs& a, cudaStream_t stream);      // fp32 CUDA cores
-// decode regime: at most 64 rows per touched group on average (uniform-routing expectation)
+// decode regime: at most kDecodeTokens rows per touched group on average (uniform-routing expectation)
 bool use_decode_ffn(int64_t rows, int G, bool grouped);
-int64_t decode_partial_slots(int64_t rows, int G, bool grouped, int d, int f);
+int64_t decode_partial_slots();  // [128][64] fp32 tiles
 int64_t decode_counter_cap(int64_t rows, int G, int d, int f);
 
 // ---- combine (combine.cu)

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 
 #include "../../include/moe.h"
 #include "common.cuh"
@@ -41,7 +42,9 @@ moe_status check_config(const moe_config* c) {
   if (c->d_model % 8 != 0 || c->d_ff % 8 != 0) return MOE_ERR_INVALID_ARG;
   if (c->top_k > c->n_experts) return MOE_ERR_INVALID_ARG;
   if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
-  if (c->gating < MOE_SOFTMAX_ALL_RENORM || c->gating > MOE_SIGMOID_TOPK_RENORM) return MOE_ERR_INVALID_ARG;
+  if (c->gating < MOE_SOFTMAX_ALL_RENORM || c->gating > MOE_SOFTMAX_ALL_NO_RENORM) return MOE_ERR_INVALID_ARG;
+  if (c->expert_act != MOE_ACT_SWIGLU && c->expert_act != MOE_ACT_GELU) return MOE_ERR_INVALID_ARG;
+  if (!(c->capacity_factor >= 0.0f) || std::isinf(c->capacity_factor)) return MOE_ERR_INVALID_ARG;
   if (c->bias_select_only != 0 && c->bias_select_only != 1) return MOE_ERR_INVALID_ARG;
   if (c->reserved != 0 || c->wait_limit_ns < 0) return MOE_ERR_INVALID_ARG;
   if (c->n_shared < 0) return MOE_ERR_INVALID_ARG;
@@ -57,6 +60,14 @@ moe_status check_config(const moe_config* c) {
 
 size_t elem_bytes(const moe_config* c) { return c->dtype == MOE_BF16 ? 2 : 4; }
 
+// Rows each expert keeps: ceil(T*k/E * capacity_factor) in double, at most T
+// (no expert is chosen twice by one token); T*k when dropless.
+int64_t capacity_rows(const moe_config* c) {
+  if (c->capacity_factor == 0.0f) return c->T * c->top_k;
+  const double cap = std::ceil((double)(c->T * c->top_k) / (double)c->n_experts * (double)c->capacity_factor);
+  return cap >= (double)c->T ? c->T : (int64_t)cap;
+}
+
 struct Carve {
   int* status;
   int32_t *ids, *counts, *offsets, *perm, *row_of, *chunk_counts;
@@ -66,6 +77,7 @@ struct Carve {
   int64_t partial_slots;
   int* counters;
   int64_t counter_cap;
+  float* aux_part;          // router penalty partial sums [kAuxMaxBlocks][E + 1]
   size_t total;
 };
 
@@ -104,9 +116,10 @@ Carve carve(const moe_config* c, void* base) {
     k.h_s = take(eb * c->T * c->d_ff_shared);
     k.y_s = take(eb * c->T * c->d_model);
   }
+  k.aux_part = static_cast<float*>(take(sizeof(float) * (size_t)kAuxMaxBlocks * (c->n_experts + 1)));
   if (decode_routed(c) || decode_shared(c)) {
-    k.partial_slots = decode_partial_slots(n, c->n_experts, true, c->d_model, c->d_ff);
-    k.partial = static_cast<float*>(take(sizeof(float) * 128 * 64 * (size_t)k.partial_slots));
+    k.partial_slots = decode_partial_slots();
+    k.partial = static_cast<float*>(take(sizeof(float) * 128 * kDecodeTokens * (size_t)k.partial_slots));
     k.counter_cap = std::max(decode_counter_cap(n, c->n_experts, c->d_model, c->d_ff),
                              c->n_shared ? decode_counter_cap(c->T, 1, c->d_model, c->d_ff_shared) : 0);
     k.counters = static_cast<int*>(take(sizeof(int) * (size_t)k.counter_cap));
@@ -146,7 +159,7 @@ uint64_t wait_limit(const moe_config* c) { return c->wait_limit_ns > 0 ? (uint64
 
 cudaError_t run_ffn(const moe_config* c, const Carve& k, const void* a, const int32_t* offsets, int G, int64_t rows,
                     int f, const void* w_gu, const void* w_d, void* h, void* y, cudaStream_t s) {
-  GroupedFfnArgs g{a, offsets, w_gu, w_d, h, y, rows, G, c->d_model, f, k.status, wait_limit(c),
+  GroupedFfnArgs g{a, offsets, w_gu, w_d, h, y, rows, G, c->d_model, f, c->expert_act, k.status, wait_limit(c),
                    k.partial, k.partial_slots, k.counters, k.counter_cap};
   if (c->dtype != MOE_BF16) return launch_grouped_ffn_f32_simt(g, s);
   if (k.partial != nullptr && use_decode_ffn(rows, G, offsets != nullptr)) return launch_grouped_ffn_bf16_decode(g, s);
@@ -163,6 +176,11 @@ extern "C" {
 size_t moe_workspace_bytes(const moe_config* cfg) {
   if (check_config(cfg) != MOE_OK) return 0;
   return carve(cfg, nullptr).total;
+}
+
+int64_t moe_expert_capacity(const moe_config* cfg) {
+  if (check_config(cfg) != MOE_OK) return -1;
+  return capacity_rows(cfg);
 }
 
 const char* moe_status_string(moe_status s) {
@@ -195,6 +213,26 @@ moe_status moe_router_topk(const moe_config* cfg, const void* x, const void* w_r
   return MOE_OK;
 }
 
+moe_status moe_router_aux_losses(const moe_config* cfg, const void* x, const void* w_router, const int32_t* counts,
+                                 float* out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+  if (!counts || !out || !aligned16(counts) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && (!x || !w_router || !aligned16(x) || !aligned16(w_router))) return MOE_ERR_INVALID_ARG;
+  if ((st = bind(ws)) != MOE_OK) return st;
+  if (cfg->T == 0) {
+    MOE_CUDA_TRY(cudaMemsetAsync(out, 0, 2 * sizeof(float), stream));
+    return MOE_OK;
+  }
+  Carve k = carve(cfg, ws);
+  // the selection itself is recomputed into the workspace and discarded
+  RouterArgs a{x, w_router, nullptr, k.ids, k.w, cfg->T, cfg->d_model, cfg->n_experts, cfg->top_k,
+               cfg->gating, cfg->bias_select_only, cfg->dtype == MOE_BF16, k.status, wait_limit(cfg), k.aux_part};
+  MOE_CUDA_TRY(launch_router_aux_losses(a, counts, out, stream));
+  return MOE_OK;
+}
+
 moe_status moe_permute(const moe_config* cfg, const int32_t* topk_ids, const void* x, int32_t* counts,
                        int32_t* offsets, int32_t* perm, int32_t* row_of, void* x_perm, void* ws, size_t ws_bytes,
                        moe_stream_t stream) {
@@ -208,7 +246,7 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_ids, const voi
   if ((st = bind(ws)) != MOE_OK) return st;
   Carve k = carve(cfg, ws);
   PermuteArgs a{topk_ids, x, counts, offsets, perm, row_of, x_perm, k.chunk_counts, cfg->T * cfg->top_k,
-                cfg->top_k, cfg->d_model, cfg->n_experts, (int)elem_bytes(cfg), k.status};
+                cfg->top_k, cfg->d_model, cfg->n_experts, (int)elem_bytes(cfg), k.status, capacity_rows(cfg)};
   MOE_CUDA_TRY(launch_permute(a, stream));
   return MOE_OK;
 }
@@ -275,7 +313,7 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
                 cfg->gating, cfg->bias_select_only, cfg->dtype == MOE_BF16, k.status, wait_limit(cfg)};
   MOE_CUDA_TRY(launch_router_topk(ra, stream));
   PermuteArgs pa{ids, x, counts, k.offsets, k.perm, k.row_of, k.x_perm, k.chunk_counts, cfg->T * cfg->top_k,
-                 cfg->top_k, cfg->d_model, cfg->n_experts, (int)elem_bytes(cfg), k.status};
+                 cfg->top_k, cfg->d_model, cfg->n_experts, (int)elem_bytes(cfg), k.status, capacity_rows(cfg)};
   MOE_CUDA_TRY(launch_permute(pa, stream));
   MOE_CUDA_TRY(run_ffn(cfg, k, k.x_perm, k.offsets, cfg->n_experts, cfg->T * cfg->top_k, cfg->d_ff, w_gate_up,
                        w_down, k.h, k.y_perm, stream));

@@ -1,20 +1,25 @@
-// Dropless dispatch: a stable counting sort of the T*k (token, slot)
-// assignments by expert, then the row gather x_perm[row] = x[perm[row] / k].
+// Dispatch: a stable counting sort of the T*k (token, slot) assignments by
+// expert, then the row gather x_perm[row] = x[perm[row] / k].
 //
 // "Mixture of Experts: why a model with 671 billion parameters uses only 37",
 // "Capacity factor: when tokens don't fit" (dropless: each expert gets exactly
-// the rows the router assigned) and "How data centres handle it" (tokens are
-// grouped by their assigned expert before the expert multiplies).
+// the rows the router assigned; with a capacity, tokens beyond an expert's
+// buffer skip it) and "How data centres handle it" (tokens are grouped by
+// their assigned expert before the expert multiplies).  The capacity rule is
+// that of "Mixture of Experts Explained: Routers, Active Parameters and VRAM"
+// (expert capacity): an expert keeps its first C assignments in token order.
 //
 // Three small kernels keep the result deterministic and stable without any
 // global atomics on positions:
 //   count   : per chunk of kChunk assignments, a shared-memory histogram
 //             -> chunk_counts[e][chunk]
 //   scan    : one block turns the histograms into counts, exclusive offsets
-//             and per-(expert, chunk) starting rows
+//             of the kept rows (min(count, C) per expert) and per-(expert,
+//             chunk) starting ranks
 //   scatter : each warp walks its slice of the chunk in order; ranks among
-//             equal experts come from __match_any_sync, so rows inside an
-//             expert follow ascending assignment index t*k+s
+//             equal experts come from __match_any_sync, so an expert's
+//             assignments are ranked in ascending index t*k+s; rank r < C
+//             lands on row offsets[e] + r, the rest are dropped (row -1)
 // and a gather kernel that moves whole rows with 16-byte loads/stores.
 #include "common.cuh"
 #include "kernels.cuh"
@@ -47,14 +52,16 @@ __global__ void __launch_bounds__(kThreads) permute_count_kernel(const int32_t* 
 // one block of kScanThreads >= E threads
 constexpr int kScanThreads = 1024;
 __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(int32_t* chunk_counts, int n_chunks, int E,
-                                                                    int32_t* counts, int32_t* offsets) {
+                                                                    int32_t* counts, int32_t* offsets,
+                                                                    int64_t capacity) {
   __shared__ int warp_sums[kScanThreads / 32];
   const int e = threadIdx.x, lane = e % 32, warp = e / 32;
   int total = 0;
   if (e < E)
     for (int b = 0; b < n_chunks; ++b) total += chunk_counts[(int64_t)e * n_chunks + b];
-  // block-wide exclusive scan of the per-expert totals
-  int incl = total;
+  const int kept = (int)min((int64_t)total, capacity);
+  // block-wide exclusive scan of the rows each expert keeps
+  int incl = kept;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const int v = __shfl_up_sync(0xffffffffu, incl, off);
@@ -72,12 +79,12 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(int32_t* chu
     warp_sums[lane] = s;  // inclusive over warps
   }
   __syncthreads();
-  const int excl = incl - total + (warp > 0 ? warp_sums[warp - 1] : 0);
+  const int excl = incl - kept + (warp > 0 ? warp_sums[warp - 1] : 0);
   if (e < E) {
     counts[e] = total;
     offsets[e] = excl;
-    if (e == E - 1) offsets[E] = excl + total;
-    int run = excl;  // per-chunk starting rows of expert e
+    if (e == E - 1) offsets[E] = excl + kept;
+    int run = 0;  // per-chunk starting ranks of expert e
     for (int b = 0; b < n_chunks; ++b) {
       const int c = chunk_counts[(int64_t)e * n_chunks + b];
       chunk_counts[(int64_t)e * n_chunks + b] = run;
@@ -88,7 +95,8 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(int32_t* chu
 
 __global__ void __launch_bounds__(kThreads) permute_scatter_kernel(const int32_t* __restrict__ ids, int64_t n,
                                                                    int E, const int32_t* __restrict__ chunk_base,
-                                                                   int n_chunks, int32_t* perm, int32_t* row_of) {
+                                                                   int n_chunks, const int32_t* __restrict__ offsets,
+                                                                   int64_t capacity, int32_t* perm, int32_t* row_of) {
   extern __shared__ int wc[];  // [kWarps][E]: per-warp counts, then per-warp next row
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   for (int i = threadIdx.x; i < kWarps * E; i += kThreads) wc[i] = 0;
@@ -104,7 +112,7 @@ __global__ void __launch_bounds__(kThreads) permute_scatter_kernel(const int32_t
     if (e >= 0 && lane == __ffs(peers) - 1) mine[e] += __popc(peers);
   }
   __syncthreads();
-  // per expert: exclusive scan over the warps, starting at this chunk's base row
+  // per expert: exclusive scan over the warps, starting at this chunk's base rank
   for (int e = threadIdx.x; e < E; e += kThreads) {
     int run = chunk_base[(int64_t)e * n_chunks + blockIdx.x];
     for (int w = 0; w < kWarps; ++w) {
@@ -123,12 +131,15 @@ __global__ void __launch_bounds__(kThreads) permute_scatter_kernel(const int32_t
     if (e >= E) e = -1;
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     int row = -1;
-    if (e >= 0) row = mine[e] + __popc(peers & lt);
+    if (e >= 0) {
+      const int rank = mine[e] + __popc(peers & lt);  // among expert e's assignments, in index order
+      if (rank < capacity) row = offsets[e] + rank;
+    }
     __syncwarp();
     if (e >= 0 && lane == __ffs(peers) - 1) mine[e] += __popc(peers);
     __syncwarp();
     if (in) {
-      row_of[i] = row;  // -1 for an id outside [0, E)
+      row_of[i] = row;  // -1 for an id outside [0, E) or a slot beyond the capacity
       if (row >= 0) perm[row] = (int32_t)i;
     }
   }
@@ -164,9 +175,10 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
   }
   permute_count_kernel<<<n_chunks, kThreads, sizeof(int) * a.E, stream>>>(a.ids, a.n_assign, a.E, a.chunk_counts,
                                                                           n_chunks, a.status);
-  permute_scan_kernel<<<1, kScanThreads, 0, stream>>>(a.chunk_counts, n_chunks, a.E, a.counts, a.offsets);
+  permute_scan_kernel<<<1, kScanThreads, 0, stream>>>(a.chunk_counts, n_chunks, a.E, a.counts, a.offsets,
+                                                      a.capacity);
   permute_scatter_kernel<<<n_chunks, kThreads, sizeof(int) * kWarps * a.E, stream>>>(
-      a.ids, a.n_assign, a.E, a.chunk_counts, n_chunks, a.perm, a.row_of);
+      a.ids, a.n_assign, a.E, a.chunk_counts, n_chunks, a.offsets, a.capacity, a.perm, a.row_of);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || a.x == nullptr || a.x_perm == nullptr) return e;
   int64_t blocks = (a.n_assign + kWarps - 1) / kWarps;

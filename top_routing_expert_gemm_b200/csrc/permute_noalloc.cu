@@ -79,7 +79,8 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
   if (scratch_address(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
   // The histogram pass writes every (expert, chunk) entry this call later
   // reads, so nothing left by an earlier call needs clearing.
+  const int64_t cap = moe_expert_capacity(cfg);
   PermuteArgs a{topk_ids, x, counts, offsets, perm, row_of, x_perm, scratch, n, cfg->top_k, cfg->d_model,
-                cfg->n_experts, cfg->dtype == MOE_BF16 ? 2 : 4, nullptr};
+                cfg->n_experts, cfg->dtype == MOE_BF16 ? 2 : 4, nullptr, cap};
   return launch_permute(a, stream) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -6,7 +6,9 @@
 // top-k-then-softmax router of "Mixture of Experts: why a model with 671
 // billion parameters uses only 37" ("The router: how a token chooses
 // experts") and its sigmoid gating ("How many experts to pick and how to
-// score them").
+// score them"); softmax probabilities kept without renormalisation as in
+// "Mixture of Experts (MoE): routing, expert parallelism, and memory" ("How
+// does MoE routing work"), the raw router probability of top-1 routing.
 //
 // One warp owns one token at a time.  Lanes split d (16-byte vector loads),
 // accumulate eight experts' dot products at once in fp32, and butterfly-reduce
@@ -33,9 +35,16 @@ struct RouterParams {
   float* wts;
   int64_t T;
   int d, E, k, gating, bias_select_only;
+  float* aux_part;  // AUX: [gridDim.x][E + 1] per-block penalty sums
 };
 
-template <typename T, bool W_SMEM, int KMAX>
+// Shared memory: logit rows [kWarps][E], with AUX the per-warp penalty sums
+// [kWarps][E] and [kWarps], then W_r [E][d] when staged.
+__host__ __device__ inline size_t router_smem_head(int E, bool aux) {
+  return sizeof(float) * kWarps * (size_t)E * (aux ? 2 : 1) + (aux ? sizeof(float) * kWarps : 0);
+}
+
+template <typename T, bool W_SMEM, int KMAX, bool AUX>
 __global__ void __launch_bounds__(kThreads) router_topk_simt_kernel(RouterParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int V = Vec16<T>::N;
@@ -45,7 +54,14 @@ __global__ void __launch_bounds__(kThreads) router_topk_simt_kernel(RouterParams
   const T* __restrict__ wg = static_cast<const T*>(p.w);
 
   float* logits = reinterpret_cast<float*>(smem) + warp * E;      // [kWarps][E]
-  T* sw = reinterpret_cast<T*>(smem + sizeof(float) * kWarps * E);  // [E][d] when staged
+  float* p_sum = reinterpret_cast<float*>(smem) + kWarps * E;     // AUX: [kWarps][E]
+  float* z_sum = p_sum + kWarps * E;                              // AUX: [kWarps]
+  T* sw = reinterpret_cast<T*>(smem + router_smem_head(E, AUX));  // [E][d] when staged
+  if (AUX) {
+    for (int i = threadIdx.x; i < kWarps * E; i += kThreads) p_sum[i] = 0.f;
+    if (threadIdx.x < kWarps) z_sum[threadIdx.x] = 0.f;
+    __syncthreads();
+  }
   if (W_SMEM) {
     const int64_t n16 = (int64_t)E * d / V;
     for (int64_t i = threadIdx.x; i < n16; i += kThreads)
@@ -98,6 +114,25 @@ __global__ void __launch_bounds__(kThreads) router_topk_simt_kernel(RouterParams
     }
     __syncwarp();
 
+    if (AUX) {
+      // penalties on the bias-free logits: softmax probabilities per expert and
+      // the squared log-sum-exp, summed over this warp's tokens in token order
+      float m = -INFINITY;
+      for (int e = lane; e < E; e += 32) m = fmaxf(m, logits[e]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      float se = 0.f;
+      for (int e = lane; e < E; e += 32) se += expf(logits[e] - m);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) se += __shfl_xor_sync(0xffffffffu, se, off);
+      const float inv = 1.0f / se;
+      for (int e = lane; e < E; e += 32) p_sum[warp * E + e] += expf(logits[e] - m) * inv;
+      if (lane == 0) {
+        const float lse = m + logf(se);
+        z_sum[warp] += lse * lse;
+      }
+    }
+
     // ---- Keep the top k of kappa = logit + bias
     TopK<KMAX> tk;
     tk.init();
@@ -137,8 +172,9 @@ __global__ void __launch_bounds__(kThreads) router_topk_simt_kernel(RouterParams
     // ---- gate weights of the selected experts
     float wsel[KMAX];
     float denom = 0.f;
-    if (p.gating == 0) {
-      // softmax over all E, keep the selected probabilities, renormalise
+    if (p.gating == 0 || p.gating == 3) {
+      // softmax over all E, keep the selected probabilities (rule 0 then
+      // renormalises them, rule 3 keeps them as they are)
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
       float z = 0.f;
@@ -174,46 +210,108 @@ __global__ void __launch_bounds__(kThreads) router_topk_simt_kernel(RouterParams
     for (int s = 0; s < KMAX; ++s) {
       if (s < k && lane == s) {
         p.ids[t * k + s] = sel_idx[s];
-        p.wts[t * k + s] = wsel[s] / denom;
+        p.wts[t * k + s] = p.gating == 3 ? wsel[s] : wsel[s] / denom;
       }
     }
     __syncwarp();
   }
+  if (AUX) {  // this block's sums, warps added in a fixed order
+    __syncthreads();
+    float* out = p.aux_part + (int64_t)blockIdx.x * (E + 1);
+    for (int e = threadIdx.x; e < E; e += kThreads) {
+      float v = 0.f;
+      for (int w = 0; w < kWarps; ++w) v += p_sum[w * E + e];
+      out[e] = v;
+    }
+    if (threadIdx.x == 0) {
+      float v = 0.f;
+      for (int w = 0; w < kWarps; ++w) v += z_sum[w];
+      out[E] = v;
+    }
+  }
 }
 
-template <typename T, bool W_SMEM>
-cudaError_t launch_t(const RouterParams& p, cudaStream_t stream) {
-  const size_t logit_bytes = sizeof(float) * kWarps * p.E;
-  const size_t smem = logit_bytes + (W_SMEM ? (size_t)p.E * p.d * sizeof(T) : 0);
+// out[0] = E * sum_e (counts[e] / sum counts) * (P_e / T), out[1] = Z / T, where
+// P_e and Z sum the per-block partials in block order.  One block.
+constexpr int kAuxThreads = 1024;
+__global__ void __launch_bounds__(kAuxThreads) router_aux_finalize_kernel(const float* __restrict__ part, int blocks,
+                                                                          int E, int64_t T,
+                                                                          const int32_t* __restrict__ counts,
+                                                                          float* out) {
+  __shared__ float red[kAuxThreads / 32];
+  float fp = 0.f;
+  for (int e = threadIdx.x; e < E; e += kAuxThreads) {
+    float pe = 0.f;
+    for (int b = 0; b < blocks; ++b) pe += part[(int64_t)b * (E + 1) + e];
+    fp += (float)counts[e] * pe;
+  }
+  // block sum of counts * P: fixed shuffle tree, then the warps in order
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) fp += __shfl_xor_sync(0xffffffffu, fp, off);
+  if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = fp;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float fptot = 0.f;
+    for (int w = 0; w < kAuxThreads / 32; ++w) fptot += red[w];
+    int64_t ctot = 0;
+    for (int e = 0; e < E; ++e) ctot += counts[e];
+    float z = 0.f;
+    for (int b = 0; b < blocks; ++b) z += part[(int64_t)b * (E + 1) + E];
+    out[0] = ctot > 0 ? (float)((double)E * (double)fptot / ((double)ctot * (double)T)) : 0.f;
+    out[1] = z / (float)T;
+  }
+}
+
+template <typename T, bool W_SMEM, bool AUX>
+cudaError_t launch_t(const RouterParams& p, int64_t max_blocks, int64_t* blocks_out, cudaStream_t stream) {
+  const size_t smem = router_smem_head(p.E, AUX) + (W_SMEM ? (size_t)p.E * p.d * sizeof(T) : 0);
   const int sms = device_sm_count();
   int64_t blocks = (p.T + kWarps - 1) / kWarps;
-  const int64_t cap = (int64_t)sms * (W_SMEM ? 2 : 8);
+  int64_t cap = (int64_t)sms * (W_SMEM ? 2 : 8);
+  if (cap > max_blocks) cap = max_blocks;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
+  if (blocks_out) *blocks_out = blocks;
   auto run = [&](auto kernel) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kernel<<<(unsigned)blocks, kThreads, smem, stream>>>(p);
     return cudaGetLastError();
   };
-  if (p.k <= 2) return run(router_topk_simt_kernel<T, W_SMEM, 2>);
-  if (p.k <= 4) return run(router_topk_simt_kernel<T, W_SMEM, 4>);
-  if (p.k <= 8) return run(router_topk_simt_kernel<T, W_SMEM, 8>);
-  return run(router_topk_simt_kernel<T, W_SMEM, 16>);
+  if (p.k <= 2) return run(router_topk_simt_kernel<T, W_SMEM, 2, AUX>);
+  if (p.k <= 4) return run(router_topk_simt_kernel<T, W_SMEM, 4, AUX>);
+  if (p.k <= 8) return run(router_topk_simt_kernel<T, W_SMEM, 8, AUX>);
+  return run(router_topk_simt_kernel<T, W_SMEM, 16, AUX>);
 }
-
-}  // namespace
 
 // W_r is staged in shared memory when it fits next to the logit rows.
 constexpr size_t kRouterSmemBudget = 160 * 1024;
 
-cudaError_t launch_router_topk_simt(const RouterArgs& a, cudaStream_t stream) {
-  RouterParams p{a.x, a.w_router, a.bias, a.ids, a.w, a.T, a.d, a.E, a.k, a.gating, a.bias_select_only};
+template <bool AUX>
+cudaError_t launch_simt(const RouterArgs& a, int64_t max_blocks, int64_t* blocks, cudaStream_t stream) {
+  RouterParams p{a.x, a.w_router, a.bias, a.ids, a.w, a.T, a.d, a.E, a.k, a.gating, a.bias_select_only, a.aux_part};
   const size_t eb = a.bf16 ? 2 : 4;
-  const bool fits = sizeof(float) * kWarps * a.E + (size_t)a.E * a.d * eb <= kRouterSmemBudget;
+  const bool fits = router_smem_head(a.E, AUX) + (size_t)a.E * a.d * eb <= kRouterSmemBudget;
   if (a.bf16)
-    return fits ? launch_t<__nv_bfloat16, true>(p, stream) : launch_t<__nv_bfloat16, false>(p, stream);
-  return fits ? launch_t<float, true>(p, stream) : launch_t<float, false>(p, stream);
+    return fits ? launch_t<__nv_bfloat16, true, AUX>(p, max_blocks, blocks, stream)
+                : launch_t<__nv_bfloat16, false, AUX>(p, max_blocks, blocks, stream);
+  return fits ? launch_t<float, true, AUX>(p, max_blocks, blocks, stream)
+              : launch_t<float, false, AUX>(p, max_blocks, blocks, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_router_topk_simt(const RouterArgs& a, cudaStream_t stream) {
+  return launch_simt<false>(a, INT64_MAX, nullptr, stream);
+}
+
+cudaError_t launch_router_aux_losses(const RouterArgs& a, const int32_t* counts, float* out, cudaStream_t stream) {
+  if (a.aux_part == nullptr) return cudaErrorInvalidValue;
+  int64_t blocks = 0;
+  cudaError_t e = launch_simt<true>(a, kAuxMaxBlocks, &blocks, stream);
+  if (e != cudaSuccess) return e;
+  router_aux_finalize_kernel<<<1, kAuxThreads, 0, stream>>>(a.aux_part, (int)blocks, a.E, a.T, counts, out);
+  return cudaGetLastError();
 }
 
 }  // namespace moe
