@@ -38,6 +38,58 @@ METRIC = "MoE-layer tokens/s (active TFLOP/s and roofline fraction alongside)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+GEMM_SOURCES = ("grouped_gemm_tc.cu", "grouped_gemm_swap.cu", "tc_primitives.cuh", "common.cuh", "kernels.cuh")
+TRAFFIC_FILE = ROOT / "profiles" / "dram_traffic.json"
+
+
+def gemm_sources_sha256() -> str:
+    """Digest of the expert-GEMM kernel sources: a DRAM-traffic record taken
+    with ncu applies only while this matches."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for name in GEMM_SOURCES:
+        h.update((ROOT / "top_routing_expert_gemm_b200" / "csrc" / name).read_bytes())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes (read + write) per step of the expert GEMMs from the committed
+    ncu record, or None when there is none or the kernels changed since."""
+    if not TRAFFIC_FILE.exists():
+        return None
+    rec = json.loads(TRAFFIC_FILE.read_text()).get(workload)
+    if not rec or rec.get("gemm_sources_sha256") != gemm_sources_sha256():
+        return None
+    return rec.get("bytes_per_step")
+
+
+def uses_decode_schedule(cfg) -> bool:
+    """The library's choice for the routed experts: the decode schedule when
+    the expected tokens per touched expert (uniform routing) is at most 64."""
+    rows = cfg.T * cfg.top_k
+    touched = max(1.0, cfg.n_experts * (1.0 - (1.0 - 1.0 / cfg.n_experts) ** rows))
+    return cfg.dtype == "bf16" and rows / touched <= 64
+
+
+def max_over_ranks(v: float, world: int, device: str = "cuda") -> float:
+    """The slowest rank's value (every rank takes part; NCCL on GPUs, gloo on CPU)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(tokens_per_rank: int, world: int, ms_max: float) -> float:
+    """Tokens/s of the whole job: every replica processed its own batch in at
+    most ``ms_max`` milliseconds (weak scaling)."""
+    return world * tokens_per_rank / (ms_max / 1000.0)
+
+
 def peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -49,18 +101,26 @@ def peaks():
 def layer_flops(cfg: synth.LayerConfig, counts: np.ndarray) -> dict:
     """Algorithmic FLOPs of one step, split by stage (rows = measured tokens per expert)."""
     rows = float(np.sum(counts))
+    mats = 3 if cfg.act == 0 else 2  # SwiGLU: gate, up, down; GELU: up, down
     router = 2.0 * cfg.T * cfg.d_model * cfg.n_experts
-    experts = 6.0 * cfg.d_model * cfg.d_ff * rows
-    shared = 6.0 * cfg.d_model * cfg.d_ff_shared * cfg.n_shared * cfg.T
+    experts = 2.0 * mats * cfg.d_model * cfg.d_ff * rows
+    shared = 2.0 * mats * cfg.d_model * cfg.d_ff_shared * cfg.n_shared * cfg.T
     return dict(router=router, experts=experts, shared=shared, total=router + experts + shared)
 
 
 def layer_bytes(cfg: synth.LayerConfig, counts: np.ndarray) -> dict:
-    """Algorithmic HBM bytes of one step: x, router, touched experts, shared experts, y."""
+    """Algorithmic HBM bytes of one step: x, router, touched experts, shared experts, y.
+    8-bit experts: one byte per weight plus one fp32 scale per weight row."""
     b = 2 if cfg.dtype == "bf16" else 4
     touched = int(np.sum(counts > 0))
-    d, f = cfg.d_model, cfg.d_ff
-    weights = touched * 3 * d * f * b + cfg.n_shared * 3 * d * cfg.d_ff_shared * b + cfg.n_experts * d * b
+    d, f, fs = cfg.d_model, cfg.d_ff, cfg.d_ff_shared
+    mats = 3 if cfg.act == 0 else 2
+    if cfg.e4m3:
+        per_expert = mats * d * f + 4 * ((mats - 1) * f + d)
+        per_shared = mats * d * fs + 4 * ((mats - 1) * fs + d)
+    else:
+        per_expert, per_shared = mats * d * f * b, mats * d * fs * b
+    weights = touched * per_expert + cfg.n_shared * per_shared + cfg.n_experts * d * b
     act = 2 * cfg.T * d * b
     return dict(weights=weights, activations=act, total=weights + act, touched=touched)
 
@@ -134,8 +194,10 @@ def config_dict(cfg: synth.LayerConfig, world: int) -> dict:
             "top_k": cfg.top_k, "d_ff": cfg.d_ff, "n_shared": cfg.n_shared, "d_ff_shared": cfg.d_ff_shared,
             "gating": cfg.gating, "zipf_s": cfg.zipf_s,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "weights": "e4m3 (per-row fp32 scales)" if cfg.e4m3 else cfg.dtype,
             "l2": "not flushed: inputs larger than L2 (expert weights %.2f GB)" % (
-                3 * cfg.n_experts * cfg.d_model * cfg.d_ff * (2 if cfg.dtype == "bf16" else 4) / 1e9)}
+                (3 if cfg.act == 0 else 2) * cfg.n_experts * cfg.d_model * cfg.d_ff
+                * (1 if cfg.e4m3 else 2 if cfg.dtype == "bf16" else 4) / 1e9)}
 
 
 def _bits_to_f64(t) -> np.ndarray:
@@ -168,7 +230,8 @@ class OracleInputs:
         self.shared = []
         for s in range(cfg.n_shared):
             gu = _bits_to_f64(dev["ws_gate_up"][s])
-            self.shared.append((gu[:fs], gu[fs:], _bits_to_f64(dev["ws_down"][s])))
+            dn = _bits_to_f64(dev["ws_down"][s])
+            self.shared.append((gu[:fs], gu[fs:], dn) if cfg.act == 0 else (gu, dn))
         per_expert_gb = 3 * cfg.d_model * cfg.d_ff * 8 / 1e9
         self.prefetched = per_expert_gb * cfg.n_experts <= prefetch_gb
         self.cache = {e: self._fetch(e) for e in range(cfg.n_experts)} if self.prefetched else None
@@ -176,7 +239,8 @@ class OracleInputs:
     def _fetch(self, e: int):
         f = self.cfg.d_ff
         gu = _bits_to_f64(self.dev["w_gate_up"][e])
-        return gu[:f], gu[f:], _bits_to_f64(self.dev["w_down"][e])
+        dn = _bits_to_f64(self.dev["w_down"][e])
+        return (gu[:f], gu[f:], dn) if self.cfg.act == 0 else (gu, dn)
 
     def expert(self, e: int):
         return self.cache[e] if self.cache is not None else self._fetch(e)
@@ -201,7 +265,7 @@ def time_oracle(oi: OracleInputs) -> float:
     cfg = oi.cfg
     t0 = time.perf_counter()
     oracle.moe_layer(oi.x, oi.wr, oi.bias, cfg.top_k, cfg.gating, oi.expert, cfg.n_experts,
-                     shared_weights=oi.shared, bias_select_only=cfg.bias_select_only)
+                     shared_weights=oi.shared, bias_select_only=cfg.bias_select_only, act=cfg.act, e4m3=cfg.e4m3)
     return time.perf_counter() - t0
 
 
@@ -259,6 +323,8 @@ def main() -> None:
     ap.add_argument("--cpu-tokens", type=int, default=128, help="tokens in the CPU-oracle baseline sample")
     ap.add_argument("--ref-tokens", type=int, default=32, help="tokens per step of --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e4m3", action="store_true",
+                    help="run the experts with 8-bit (FP8 E4M3) weights, quantised on the GPU from the bf16 ones")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -273,9 +339,13 @@ def main() -> None:
         if field not in ("d_model", "d_ff", "n_experts", "top_k", "d_ff_shared"):
             ap.error(f"--set: unknown field {field}")
         cfg = cfg.replace(**{field: int(val)})
-    if args.set or args.T is not None or args.zipf is not None:
+    if args.e4m3:
+        if cfg.dtype != "bf16":
+            ap.error("--e4m3 needs a bf16 workload")
+        cfg = cfg.replace(e4m3=True)
+    if args.set or args.T is not None or args.zipf is not None or args.e4m3:
         cfg = cfg.replace(name=f"{cfg.name}[T={cfg.T},d={cfg.d_model},f={cfg.d_ff},E={cfg.n_experts},"
-                               f"k={cfg.top_k},zipf={cfg.zipf_s}]")
+                               f"k={cfg.top_k},zipf={cfg.zipf_s}" + (",e4m3]" if cfg.e4m3 else "]"))
 
     if args.impl == "reference":
         run_reference(args, cfg)
@@ -303,9 +373,18 @@ def main() -> None:
                                         name, "cuda")
     bias_np = synth.zipf_bias(cfg)
     bias = torch.from_numpy(bias_np).cuda() if bias_np is not None else None
+    wfmt = moe.MOE_W_E4M3 if cfg.e4m3 else moe.MOE_W_NATIVE
+    if cfg.e4m3:  # the expert weights as the library's 8-bit blobs, quantised on the GPU
+        for name in ("w_gate_up", "w_down", "ws_gate_up", "ws_down"):
+            if name in dev:
+                src = dev[name]
+                rows = src.numel() // src.shape[-1]
+                blob = torch.empty(moe.moe_e4m3_weight_bytes(rows, src.shape[-1]), dtype=torch.uint8, device="cuda")
+                moe.moe_quantize_e4m3(src, rows, src.shape[-1], blob)
+                dev[name + "_q"] = blob  # the bf16 values stay for the CPU oracle, which quantises them itself
     c = moe.make_config(cfg.T, cfg.d_model, cfg.n_experts, cfg.top_k, cfg.d_ff,
                         moe.MOE_BF16 if cfg.dtype == "bf16" else moe.MOE_F32, cfg.gating, cfg.n_shared,
-                        cfg.d_ff_shared, cfg.bias_select_only)
+                        cfg.d_ff_shared, cfg.bias_select_only, expert_act=cfg.act, weight_format=wfmt)
     tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     T, d, k, E = cfg.T, cfg.d_model, cfg.top_k, cfg.n_experts
     ws_bytes = moe.moe_workspace_bytes(c)
@@ -316,20 +395,15 @@ def main() -> None:
     counts = torch.empty(E, dtype=torch.int32, device="cuda")
     stream = torch.cuda.current_stream()
 
+    q = "_q" if cfg.e4m3 else ""  # the expert weights the kernels read
+
     def step():
-        moe.moe_forward(c, dev["x"], dev["w_router"], bias, dev["w_gate_up"], dev["w_down"], dev.get("ws_gate_up"),
-                        dev.get("ws_down"), y, ids, w, counts, ws, ws_bytes, stream)
+        moe.moe_forward(c, dev["x"], dev["w_router"], bias, dev["w_gate_up" + q], dev["w_down" + q],
+                        dev.get("ws_gate_up" + q), dev.get("ws_down" + q), y, ids, w, counts, ws, ws_bytes, stream)
 
     def barrier():
         if world > 1:
             dist.barrier()
-
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     for _ in range(args.warmup):
         step()
@@ -350,7 +424,7 @@ def main() -> None:
         ev1.record(stream)
         torch.cuda.synchronize()
         barrier()
-    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world)
     clocks = clk.summary()
 
     # ---- same step as its four C-ABI stages, events between them (per-stage split, roofline)
@@ -364,7 +438,8 @@ def main() -> None:
     stage_names = ["router_topk", "permute", "grouped_ffn"] + (["shared_ffn"] if cfg.n_shared else []) + ["combine"]
     if cfg.n_shared:
         # the always-on expert as one group over all T tokens
-        c_s = moe.make_config(T, d, 1, 1, cfg.d_ff_shared, c.dtype, cfg.gating)
+        c_s = moe.make_config(T, d, 1, 1, cfg.d_ff_shared, c.dtype, cfg.gating, expert_act=cfg.act,
+                              weight_format=wfmt)
         ws_s_bytes = moe.moe_workspace_bytes(c_s)
         ws_s = torch.zeros(ws_s_bytes, dtype=torch.uint8, device="cuda")
         off_s = torch.tensor([0, T], dtype=torch.int32, device="cuda")
@@ -385,11 +460,11 @@ def main() -> None:
         mark()
         moe.moe_permute(c, ids2, dev["x"], counts2, offsets, perm, row_of, x_perm, ws, ws_bytes, stream)
         mark()
-        moe.moe_grouped_ffn(c, x_perm, offsets, dev["w_gate_up"], dev["w_down"], y_perm, ws, ws_bytes, stream)
+        moe.moe_grouped_ffn(c, x_perm, offsets, dev["w_gate_up" + q], dev["w_down" + q], y_perm, ws, ws_bytes, stream)
         mark()
         if cfg.n_shared:
-            moe.moe_grouped_ffn(c_s, dev["x"], off_s, dev["ws_gate_up"], dev["ws_down"], y_sh, ws_s, ws_s_bytes,
-                                stream)
+            moe.moe_grouped_ffn(c_s, dev["x"], off_s, dev["ws_gate_up" + q], dev["ws_down" + q], y_sh, ws_s,
+                                ws_s_bytes, stream)
             mark()
         moe.moe_combine(c, y_perm, row_of, w2, y_sh if cfg.n_shared else None, y, stream)
         mark()
@@ -411,8 +486,8 @@ def main() -> None:
 
     def e2e_step():
         x_in.copy_(x_host, non_blocking=True)
-        moe.moe_forward(c, x_in, dev["w_router"], bias, dev["w_gate_up"], dev["w_down"], dev.get("ws_gate_up"),
-                        dev.get("ws_down"), y, ids, w, counts, ws, ws_bytes, stream)
+        moe.moe_forward(c, x_in, dev["w_router"], bias, dev["w_gate_up" + q], dev["w_down" + q],
+                        dev.get("ws_gate_up" + q), dev.get("ws_down" + q), y, ids, w, counts, ws, ws_bytes, stream)
         y_host.copy_(y, non_blocking=True)
 
     for _ in range(args.warmup):
@@ -426,12 +501,12 @@ def main() -> None:
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
 
     pk, pk_kind = peaks()
     fl = layer_flops(cfg, counts_np)
     by = layer_bytes(cfg, counts_np)
-    tokens_per_s = world * T / (ms / 1000.0)
+    tokens_per_s = replica_throughput(T, world, ms)
     active_tflops = world * fl["total"] / (ms / 1000.0) / 1e12
     # dominant kernel: the grouped expert GEMMs (tcgen05), timed as the moe_grouped_ffn stage
     g_ms = stage_ms["grouped_ffn"] + stage_ms.get("shared_ffn", 0.0)
@@ -442,23 +517,33 @@ def main() -> None:
         roof = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": gbs / pk["hbm_gbs"], "traffic": None}
     else:
-        roof = {"bound": "tensor", "achieved": gemm_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": gemm_tflops / pk["bf16_tflops"], "traffic": None}
-    roof["kernel"] = ("grouped_gemm_tc: the GEMM-1+SwiGLU and GEMM-2 launches of moe_grouped_ffn"
+        # 8-bit experts: the measured bf16 peak x 2, the nominal dense fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s)
+        tpk = pk["bf16_tflops"] * (2.0 if cfg.e4m3 else 1.0)
+        roof = {"bound": "tensor", "achieved": gemm_tflops, "peak": tpk, "unit": "TFLOP/s",
+                "frac": gemm_tflops / tpk, "traffic": None}
+    if cfg.dtype != "bf16":
+        kname = "grouped_gemm_f32_kernel (CUDA cores)"
+    elif uses_decode_schedule(cfg):
+        kname = "grouped_gemm_swap_kernel, decode schedule (weight rows as M, reductions split evenly over the CTAs)"
+    else:
+        kname = "grouped_gemm_tc_kernel (token rows as M)"
+    roof["kernel"] = (kname + ": the GEMM-1 and GEMM-2 launches of moe_grouped_ffn"
                       + (" (routed and shared experts)" if cfg.n_shared else ""))
-    roof["peak_source"] = pk_kind
+    roof["traffic"] = recorded_traffic(cfg.name)
+    roof["peak_source"] = pk_kind + (" bf16 x 2 (nominal fp8/bf16 dense ratio)" if cfg.e4m3 and not decode else "")
     line = {
         "metric": METRIC,
         "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": cfg.dtype, "data": "synthetic (seeded counter-based generator; random-init weights)",
+        "dtype": "e4m3" if cfg.e4m3 else cfg.dtype,
+        "data": "synthetic (seeded counter-based generator; random-init weights)",
         "config": config_dict(cfg, world),
         "active_tflops": active_tflops,
         "stage_ms": stage_ms,
         "roofline": roof,
         "experts_touched": by["touched"],
         "clocks": clocks,
-        "e2e": {"value": world * T / (e2e_ms / 1000.0), "unit": "tokens/s",
+        "e2e": {"value": replica_throughput(T, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * d * x_host.element_size(),
                 "d2h_bytes_per_step": T * d * y_host.element_size()},
         "gpu_launches": args.steps * (8 if cfg.n_shared == 0 else 10),

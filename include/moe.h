@@ -114,6 +114,22 @@ typedef enum {
   MOE_ACT_GELU = 1
 } moe_expert_act;
 
+typedef enum {
+  /* expert weights in dtype (bf16 or fp32) */
+  MOE_W_NATIVE = 0,
+  /* 8-bit experts: every expert weight tensor (w_gate_up, w_down, ws_gate_up,
+     ws_down) is an E4M3 blob made by moe_quantize_e4m3: FP8 E4M3 codes of the
+     [rows, cols] matrix (rows = E*2f or E*f, resp. E*d; cols = d, resp. f),
+     then at byte offset align256(rows*cols) one fp32 scale per row.  The
+     expert inputs (x_perm, the shared expert's x) and h are quantised per
+     token row the same way inside the call; accumulation is fp32, h and the
+     outputs stay bf16.  Requires dtype MOE_BF16 and d_model, d_ff, d_ff_shared
+     multiples of 16.  The pages name 8-bit experts ("Mixture of Experts: why
+     a model...", "How data centres handle it") without fixing a scheme; per-
+     row absolute-max scaling to E4M3 is the one used here.                 */
+  MOE_W_E4M3 = 1
+} moe_weight_format;
+
 typedef struct {
   int64_t T;                /* tokens                                          */
   int32_t d_model;          /* d                                               */
@@ -136,7 +152,7 @@ typedef struct {
                                capacity).  A dropped slot adds nothing to its
                                token's output; the other slots keep their
                                weights.                                        */
-  int32_t reserved;         /* must be 0                                       */
+  int32_t weight_format;    /* moe_weight_format of the expert weights         */
 } moe_config;
 
 /* Bytes of scratch every entry point below accepts for this config
@@ -146,6 +162,18 @@ size_t moe_workspace_bytes(const moe_config* cfg);
 
 /* Static, NUL-terminated description of a status code. */
 const char* moe_status_string(moe_status s);
+
+/* Bytes of an E4M3 weight blob for a [rows, cols] matrix: align256(rows*cols)
+   code bytes, then rows fp32 scales; 0 when cols is not a positive multiple
+   of 16. */
+size_t moe_e4m3_weight_bytes(int64_t rows, int64_t cols);
+
+/* Quantise a bf16 [rows, cols] row-major matrix into an E4M3 blob (see
+   MOE_W_E4M3): per row s = max|w| / 448 (1 for a zero row), codes =
+   E4M3(w / s) rounded to nearest even with saturation.  blob: device,
+   256-byte aligned, moe_e4m3_weight_bytes(rows, cols) bytes.  Asynchronous
+   on stream; allocates nothing. */
+moe_status moe_quantize_e4m3(const void* src, int64_t rows, int32_t cols, void* blob, moe_stream_t stream);
 
 /* Rows each expert keeps: ceil(T*k/E * capacity_factor) evaluated in double
    (capped at T, which no expert can exceed) when capacity_factor > 0, T*k

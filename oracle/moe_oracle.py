@@ -83,7 +83,8 @@ ACT_GELU = 1     # plain expert, two matrices (w_up [f, d], w_down [d, f])
 __all__ = [
     "SOFTMAX_ALL_RENORM", "SOFTMAX_TOPK", "SIGMOID_TOPK_RENORM", "SOFTMAX_ALL_NO_RENORM",
     "ACT_SWIGLU", "ACT_GELU", "gelu", "gelu_expert", "expert_capacity", "dropped_slots",
-    "balance_loss", "router_z_loss", "logsumexp",
+    "balance_loss", "router_z_loss", "logsumexp", "E4M3_MAX", "e4m3_round", "e4m3_decode",
+    "quantize_rows_e4m3", "round_bf16", "e4m3_expert",
     "router_logits", "selection_key", "topk_select", "topk_gap", "softmax", "sigmoid",
     "gate_weights", "Routing", "route", "dispatch", "silu", "swiglu_expert", "moe_layer",
     "occupancy_closed_form", "occupancy_monte_carlo", "expert_params", "moe_layer_params",
@@ -297,7 +298,8 @@ def moe_layer(x: np.ndarray, w_router: np.ndarray | None, bias: np.ndarray | Non
               bias_select_only: int = 0, ids: np.ndarray | None = None,
               decision_dtype=np.float32, act: int = ACT_SWIGLU,
               capacity: int | None = None,
-              keep: np.ndarray | None = None) -> tuple[np.ndarray, Routing | None, np.ndarray]:
+              keep: np.ndarray | None = None,
+              e4m3: bool = False) -> tuple[np.ndarray, Routing | None, np.ndarray]:
     """Sparse MoE sublayer output for the tokens ``x`` [T, d].
 
     Router -> top-k -> per-expert loop -> weighted sum, as in [TUR]'s
@@ -317,6 +319,9 @@ def moe_layer(x: np.ndarray, w_router: np.ndarray | None, bias: np.ndarray | Non
     layer; the residual connection that carries it lies outside this sublayer).
     ``keep`` ([T, k] bool) gives the kept slots directly, for evaluating a
     subset of a batch whose drops were decided over the whole batch.
+
+    ``e4m3``: experts run with 8-bit weights and activations
+    (:func:`e4m3_expert`).
 
     Forced routing: when ``ids`` is given the selection is taken from it and
     only the gate weights and expert outputs are recomputed (``w_router``
@@ -340,6 +345,8 @@ def moe_layer(x: np.ndarray, w_router: np.ndarray | None, bias: np.ndarray | Non
             keep = (row_of >= 0).reshape(ids_.shape)
 
     def ffn(xr, wts):
+        if e4m3:
+            return e4m3_expert(xr, wts, act)
         return swiglu_expert(xr, *wts) if act == ACT_SWIGLU else gelu_expert(xr, *wts)
 
     y = np.zeros_like(x)
@@ -351,6 +358,87 @@ def moe_layer(x: np.ndarray, w_router: np.ndarray | None, bias: np.ndarray | Non
     for wts in shared_weights:
         y += ffn(x, wts)
     return y, r, w
+
+
+# ---------------------------------------------------------------- 8-bit experts
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(code: int) -> float:
+    """Value of an FP8 E4M3 code (1 sign bit, 4 exponent bits with bias 7,
+    3 mantissa bits; exponent 0 is subnormal; S.1111.111 is NaN, so the
+    largest finite value is 1.75 * 2^8 = 448)."""
+    sgn = -1.0 if code & 0x80 else 1.0
+    ex = (code >> 3) & 0xF
+    man = code & 0x7
+    if ex == 0xF and man == 0x7:
+        return float("nan")
+    if ex == 0:
+        return sgn * man / 8.0 * 2.0 ** -6
+    return sgn * (1.0 + man / 8.0) * 2.0 ** (ex - 7)
+
+
+def e4m3_round(v) -> np.ndarray:
+    """Nearest FP8 E4M3 value (ties to even), saturating at +-448, as float64.
+
+    Normal binades [2^e, 2^(e+1)) for e in -6..8 hold 8 values spaced
+    2^(e-3); below 2^-6 the subnormals are spaced 2^-9.  ``np.rint`` rounds
+    half to even; scaling by a power of two is exact."""
+    a = np.abs(np.asarray(v, dtype=np.float64))
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))   # a = m * 2^ex, m in [0.5, 1)
+    e = np.clip(ex - 1, -6, 8)
+    step = np.ldexp(1.0, e - 3)
+    q = np.minimum(np.rint(a / step) * step, E4M3_MAX)
+    return np.copysign(q, np.asarray(v, dtype=np.float64))
+
+
+def quantize_rows_e4m3(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Per-row FP8 E4M3 quantisation with a float32 scale: ``s = max|x| / 448``
+    (1 for an all-zero row), ``q = e4m3(float32(x / s))``, so that x ~ q * s.
+    The pages name 8-bit experts without a scheme; this per-row absolute-max
+    scaling is the plainest one.  The decisions are taken in float32, the
+    precision of the kernels (x is exact in float32: bf16 or fp32 storage).
+    Returns (q as float64 values, s as float64)."""
+    x32 = np.asarray(x, dtype=np.float32)
+    amax = np.max(np.abs(x32), axis=1)
+    s = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    q = e4m3_round((x32 / s[:, None]).astype(np.float32))
+    return q, s.astype(np.float64)
+
+
+def round_bf16(v: np.ndarray) -> np.ndarray:
+    """float64 -> float32 -> bfloat16, each step to nearest with ties to even
+    (how a kernel stores an fp32 result as bf16), returned as float64."""
+    f = np.ascontiguousarray(np.asarray(v, dtype=np.float64).astype(np.float32))
+    b = f.view(np.uint32).astype(np.uint64)
+    b = ((b + 0x7FFF + ((b >> 16) & 1)) >> 16) << 16
+    return b.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def e4m3_expert(xr: np.ndarray, weights, act: int) -> np.ndarray:
+    """One expert with 8-bit weights and activations.
+
+    The pages name 8-bit and 4-bit experts ([TUR] "How data centres handle
+    it", [AFD] "What mixture of experts costs in memory") but fix no scheme;
+    the plainest one is used: every weight row (output channel) and every
+    token row of the expert's input is quantised to FP8 E4M3 with its own
+    scale (:func:`quantize_rows_e4m3`), the products are exact and summed
+    without rounding, the hidden activation h is stored as bf16 (the
+    kernels' storage) and quantised per token row the same way before the
+    down projection.  xr [n, d] (the stored bf16 values); weights as in
+    :func:`moe_layer`."""
+    def deq(m):
+        q, s = quantize_rows_e4m3(m)
+        return q * s[:, None]
+
+    xd = deq(xr)
+    if act == ACT_SWIGLU:
+        wg, wu, wd = weights
+        h = silu(xd @ deq(wg).T) * (xd @ deq(wu).T)
+    else:
+        wu, wd = weights
+        h = gelu(xd @ deq(wu).T)
+    return deq(round_bf16(h)) @ deq(wd).T
 
 
 # ---------------------------------------------------------------- router penalties

@@ -184,6 +184,7 @@ class LayerConfig:
     seed: int = 1000
     act: int = 0           # 0: SwiGLU expert (gate+up rows), 1: GELU expert (up rows only)
     capacity_factor: float = 0.0  # 0: dropless
+    e4m3: bool = False     # expert weights run as FP8 E4M3 (quantised from the generated bf16 values)
 
     def replace(self, **kw) -> "LayerConfig":
         return dataclasses.replace(self, **kw)

@@ -32,7 +32,17 @@ def moe_cfg(cfg: synth.LayerConfig, T: int | None = None, wait_limit_ns: int = 0
     return moe.make_config(cfg.T if T is None else T, cfg.d_model, cfg.n_experts, cfg.top_k, cfg.d_ff,
                            moe.MOE_BF16 if cfg.dtype == "bf16" else moe.MOE_F32, cfg.gating,
                            cfg.n_shared, cfg.d_ff_shared, cfg.bias_select_only, wait_limit_ns,
-                           expert_act=cfg.act, capacity_factor=cfg.capacity_factor)
+                           expert_act=cfg.act, capacity_factor=cfg.capacity_factor,
+                           weight_format=moe.MOE_W_E4M3 if cfg.e4m3 else moe.MOE_W_NATIVE)
+
+
+def e4m3_blob(w: torch.Tensor) -> torch.Tensor:
+    """The library's E4M3 blob of a bf16 weight tensor [..., rows, cols] (made on the GPU)."""
+    cols = w.shape[-1]
+    rows = w.numel() // cols
+    blob = torch.empty(moe.moe_e4m3_weight_bytes(rows, cols), dtype=torch.uint8, device=w.device)
+    moe.moe_quantize_e4m3(w, rows, cols, blob)
+    return blob
 
 
 def capacity_of(cfg: synth.LayerConfig) -> int | None:
@@ -76,6 +86,10 @@ def make_inputs(cfg: synth.LayerConfig, device="cuda", host_limit: int = 1 << 24
             dev[name] = synth.device_tensor(cfg, name, device)
     bias = synth.zipf_bias(cfg)
     dev["bias"] = torch.from_numpy(bias).to(device) if bias is not None else None
+    if cfg.e4m3:  # the kernels read the 8-bit blobs; the oracle quantises the bf16 values itself
+        for name in ("w_gate_up", "w_down", "ws_gate_up", "ws_down"):
+            if name in dev:
+                dev[name + "_q"] = e4m3_blob(dev[name])
     return Inputs(cfg, dev, bias, on_host)
 
 
@@ -144,8 +158,9 @@ def run_forward(inp: Inputs, wait_limit_ns: int = 0):
     w = torch.empty(T, k, dtype=torch.float32, device="cuda")
     counts = torch.empty(E, dtype=torch.int32, device="cuda")
     ws = torch.empty(max(256, moe.moe_workspace_bytes(c)), dtype=torch.uint8, device="cuda")
-    moe.moe_forward(c, dev["x"], dev["w_router"], dev["bias"], dev["w_gate_up"], dev["w_down"],
-                    dev.get("ws_gate_up"), dev.get("ws_down"), y, ids, w, counts, ws)
+    q = "_q" if cfg.e4m3 else ""
+    moe.moe_forward(c, dev["x"], dev["w_router"], dev["bias"], dev["w_gate_up" + q], dev["w_down" + q],
+                    dev.get("ws_gate_up" + q), dev.get("ws_down" + q), y, ids, w, counts, ws)
     st = moe.moe_device_status(ws)
     torch.cuda.synchronize()
     return dict(y=y, ids=ids, w=w, counts=counts, ws=ws, status=st)
@@ -209,7 +224,7 @@ def check_forward(inp: Inputs, out: dict, n_sample: int | None = None) -> dict:
     tokens = np.arange(T) if n_sample is None else sample_tokens(T, n_sample)
     y_ref, _, _ = oracle.moe_layer(x_all[tokens], wr, bias, k, cfg.gating, ow.routed, E,
                                    shared_weights=ow.shared(), bias_select_only=cfg.bias_select_only,
-                                   ids=gpu_ids[tokens], act=cfg.act, keep=keep[tokens])
+                                   ids=gpu_ids[tokens], act=cfg.act, keep=keep[tokens], e4m3=cfg.e4m3)
     y = device_to_host_f64(out["y"][torch.from_numpy(tokens).cuda()])
     err = rel_err(y, y_ref)
     assert err <= TOL[cfg.dtype], f"relative error {err:.3e} > {TOL[cfg.dtype]}"

@@ -89,6 +89,7 @@ def test_config_struct_layout():
     assert moe.MoeConfig.expert_act.offset == 44
     assert moe.MoeConfig.wait_limit_ns.offset == 48
     assert moe.MoeConfig.capacity_factor.offset == 56
+    assert moe.MoeConfig.weight_format.offset == 60
 
 
 def test_expert_capacity_host_arithmetic(L):

@@ -57,6 +57,16 @@ SMALL = {
     "gelu_capacity_shared": synth.LayerConfig("gelu_capacity_shared", 200, 256, 16, 4, 192, "bf16",
                                               synth.SOFTMAX_ALL_NO_RENORM, n_shared=1, d_ff_shared=256, act=1,
                                               zipf_s=1.0, capacity_factor=0.8, seed=31),
+    # 8-bit (E4M3) experts: large-batch and decode schedules, shared expert, GELU
+    "e4m3_mixtral_like": synth.LayerConfig("e4m3_mixtral_like", 300, 512, 8, 2, 640, "bf16", synth.SOFTMAX_TOPK,
+                                           e4m3=True, seed=32),
+    "e4m3_decode": synth.LayerConfig("e4m3_decode", 5, 1024, 8, 2, 1536, "bf16", synth.SOFTMAX_TOPK, e4m3=True,
+                                     seed=33),
+    "e4m3_deepseek_like": synth.LayerConfig("e4m3_deepseek_like", 257, 512, 64, 8, 256, "bf16",
+                                            synth.SIGMOID_TOPK_RENORM, n_shared=1, d_ff_shared=384, zipf_s=1.0,
+                                            bias_select_only=1, e4m3=True, seed=34),
+    "e4m3_gelu": synth.LayerConfig("e4m3_gelu", 200, 256, 16, 2, 320, "bf16", synth.SOFTMAX_ALL_RENORM, act=1,
+                                   e4m3=True, seed=35),
 }
 
 
@@ -328,3 +338,66 @@ def test_router_aux_losses(dtype, E, k, d, T):
     assert abs(got[0] - ref[0]) <= 1e-4 * abs(ref[0]), (got, ref)
     assert abs(got[1] - ref[1]) <= 1e-4 * abs(ref[1]), (got, ref)
     assert np.isnan(got[2]) and np.isnan(got[3])  # nothing written past out[1]
+
+
+# ------------------------------------------------------------------ 8-bit experts
+def test_quantize_e4m3_matches_the_oracle_bit_for_bit():
+    """Codes and scales of moe_quantize_e4m3 equal the oracle's per-row E4M3
+    quantisation of the same bf16 values (the rounding decisions are taken
+    in float32 on both sides): values exactly, scales exactly."""
+    rng = np.random.default_rng(40)
+    rows, cols = 70, 272
+    w = rng.standard_normal((rows, cols)).astype(np.float32)
+    w[3] = 0.0
+    w[5] *= 1e-4
+    w[6] *= 3e3
+    w[7, 11] = 1e6  # one outlier dominates its row's scale
+    wt = torch.from_numpy(w).to(torch.bfloat16).cuda()
+    blob = H.e4m3_blob(wt)
+    assert blob.numel() == moe.moe_e4m3_weight_bytes(rows, cols) == (rows * cols + 255) // 256 * 256 + 4 * rows
+    codes = blob[: rows * cols].cpu().numpy().reshape(rows, cols)
+    off = (rows * cols + 255) // 256 * 256
+    scales = blob[off: off + 4 * rows].cpu().numpy().view(np.float32).astype(np.float64)
+    table = np.array([oracle.e4m3_decode(c) for c in range(256)])
+    q_ref, s_ref = oracle.quantize_rows_e4m3(H.device_to_host_f64(wt))
+    assert np.array_equal(scales, s_ref)
+    assert np.array_equal(table[codes], q_ref)
+
+
+@pytest.mark.parametrize("act", [0, 1])
+@pytest.mark.parametrize("sizes,d,f", [
+    ([0, 1, 127, 129, 300, 0, 256], 256, 384),   # large-batch schedule
+    ([3, 0, 40, 1], 1024, 1536),                  # decode schedule, units cut across CTAs
+    ([600, 17], 272, 208),                        # partial weight blocks
+])
+def test_grouped_ffn_e4m3_against_the_oracle(act, sizes, d, f):
+    """8-bit experts through moe_grouped_ffn: weights quantised on the GPU,
+    activations and h inside the call; the oracle quantises the same bf16
+    values itself (e4m3_expert).  Tolerance: the bf16 one."""
+    rng = np.random.default_rng(sum(sizes) + d + f + act)
+    G = len(sizes)
+    rows = int(sum(sizes))
+    offs = _ragged_offsets(sizes)
+    m = 2 if act == 0 else 1
+    a = torch.from_numpy(rng.standard_normal((rows, d)).astype(np.float32)).to(torch.bfloat16).cuda()
+    wgu = torch.from_numpy((rng.standard_normal((G, m * f, d)) / np.sqrt(d)).astype(np.float32)).to(torch.bfloat16)
+    wd = torch.from_numpy((rng.standard_normal((G, d, f)) / np.sqrt(f)).astype(np.float32)).to(torch.bfloat16)
+    wgu, wd = wgu.cuda(), wd.cuda()
+    y = torch.full((rows, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    cfg = synth.LayerConfig("g", rows, d, G, 1, f, "bf16", 0, act=act, e4m3=True)
+    c = H.moe_cfg(cfg)
+    ws = torch.zeros(moe.moe_workspace_bytes(c), dtype=torch.uint8, device="cuda")
+    moe.moe_grouped_ffn(c, a, torch.from_numpy(offs).cuda(), H.e4m3_blob(wgu), H.e4m3_blob(wd), y, ws)
+    assert moe.moe_device_status(ws) == 0
+    A = H.device_to_host_f64(a)
+    WGU = H.device_to_host_f64(wgu)
+    WD = H.device_to_host_f64(wd)
+    ref = np.zeros((rows, d))
+    for g in range(G):
+        r0, r1 = offs[g], offs[g + 1]
+        if r1 > r0:
+            wts = (WGU[g, :f], WGU[g, f:], WD[g]) if act == 0 else (WGU[g], WD[g])
+            ref[r0:r1] = oracle.e4m3_expert(A[r0:r1], wts, act)
+    got = H.device_to_host_f64(y)
+    assert not np.any(np.isnan(got))
+    assert H.rel_err(got, ref) <= H.TOL["bf16"]

@@ -544,3 +544,133 @@ def test_router_z_loss_closed_forms():
     l = np.array([[0.0, math.log(3.0)], [1.0, 1.0]])
     ref = (math.log(1 + 3) ** 2 + (1 + math.log(2)) ** 2) / 2
     assert abs(oracle.router_z_loss(l) - ref) <= 1e-14
+
+
+# ------------------------------------------------------------------ FP8 E4M3 quantisation
+def _e4m3_table():
+    """All finite E4M3 values from the bit layout (sign, 4-bit exponent with
+    bias 7, 3-bit mantissa, subnormals at exponent 0, NaN at S.1111.111)."""
+    vals = []
+    for code in range(256):
+        v = oracle.e4m3_decode(code)
+        if not math.isnan(v):
+            vals.append(v)
+    return np.array(sorted(set(vals)))
+
+
+def test_e4m3_decode_landmarks():
+    """448 largest finite, 2^-9 smallest subnormal, 2^-6 smallest normal, 1.0 = 0x38."""
+    assert oracle.e4m3_decode(0x7E) == 448.0 and math.isnan(oracle.e4m3_decode(0x7F))
+    assert oracle.e4m3_decode(0x01) == 2.0 ** -9 and oracle.e4m3_decode(0x08) == 2.0 ** -6
+    assert oracle.e4m3_decode(0x38) == 1.0 and oracle.e4m3_decode(0xB8) == -1.0
+    assert len(_e4m3_table()) == 253  # 254 finite codes, +0 and -0 equal
+
+
+def test_e4m3_round_is_nearest_representable_ties_to_even():
+    """Brute force against the decoded table: every value maps to its nearest
+    representable neighbour, midpoints to the one with an even mantissa, the
+    table onto itself, and anything beyond 448 saturates."""
+    table = _e4m3_table()
+    assert np.array_equal(oracle.e4m3_round(table), table)
+    rng = np.random.default_rng(3)
+    v = np.concatenate([rng.standard_normal(4000) * 10.0, rng.standard_normal(2000) * 0.01,
+                        (table[1:] + table[:-1]) / 2])       # every midpoint
+    got = oracle.e4m3_round(v)
+    for x, g in zip(v, got):
+        d = np.abs(table - x)
+        near = table[d == d.min()]
+        if x > 448.0 or x < -448.0:
+            assert g == np.sign(x) * 448.0
+        elif len(near) == 1:
+            assert g == near[0], x
+        else:  # a tie: the even mantissa (its code has bit 0 clear)
+            even = [t for t in near if int(round(abs(t) / _ulp(abs(t)))) % 2 == 0]
+            assert g == even[0], (x, near)
+
+
+def _ulp(a: float) -> float:
+    if a < 2.0 ** -6:
+        return 2.0 ** -9
+    return 2.0 ** (math.floor(math.log2(a)) - 3)
+
+
+def test_quantize_rows_reconstructs_within_half_a_step():
+    """x ~ q * s with |x - q s| <= half an E4M3 step of x / s; the row's largest
+    magnitude maps to exactly 448; a zero row gets scale 1."""
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((20, 300)).astype(np.float32)
+    x[3] = 0.0
+    q, s = oracle.quantize_rows_e4m3(x)
+    assert s[3] == 1.0 and np.all(q[3] == 0.0)
+    for r in range(20):
+        if r == 3:
+            continue
+        assert np.max(np.abs(q[r])) == 448.0
+        y = x[r].astype(np.float64) / s[r]
+        for a, b in zip(y, q[r]):
+            assert abs(a - b) <= 0.5 * _ulp(abs(a)) * (1 + 1e-6) + 1e-12
+
+
+def test_round_bf16_is_nearest_of_the_two_neighbours():
+    """Brute force: the bf16 result is the closer of the two bf16 values around
+    the float32 value (ties to the one whose last mantissa bit is 0)."""
+    rng = np.random.default_rng(11)
+    v = np.concatenate([rng.standard_normal(3000), np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -2.5])])
+    got = oracle.round_bf16(v)
+    for x, g in zip(v.astype(np.float32).astype(np.float64), got):
+        m, e = math.frexp(abs(x))            # |x| = m 2^e, m in [0.5, 1)
+        step = 2.0 ** (e - 8)                # bf16 keeps 8 significant bits
+        lo = math.floor(abs(x) / step) * step
+        hi = lo + step
+        if abs(x) - lo < hi - abs(x):
+            want = lo
+        elif abs(x) - lo > hi - abs(x):
+            want = hi
+        else:
+            want = lo if int(lo / step) % 2 == 0 else hi
+        assert g == math.copysign(want, x), (x, g, want)
+
+
+def _e4m3_layer_inputs(rng, n=6, d=40, f=24):
+    x = rng.standard_normal((n, d))
+    wg = rng.standard_normal((f, d)) / np.sqrt(d)
+    wu = rng.standard_normal((f, d)) / np.sqrt(d)
+    wd = rng.standard_normal((d, f)) / np.sqrt(f)
+    return x, (wg, wu, wd)
+
+
+def test_e4m3_expert_scales_are_per_token_and_per_output_channel():
+    """Changing one token row leaves the other rows' outputs bit-identical (no
+    per-tensor activation scale); scaling one down-projection row by 2^k
+    scales exactly that output column by 2^k (its codes are unchanged, only
+    its scale moves) and leaves the others bit-identical (no per-input-column
+    weight scale)."""
+    rng = np.random.default_rng(21)
+    x, (wg, wu, wd) = _e4m3_layer_inputs(rng)
+    base = oracle.e4m3_expert(x, (wg, wu, wd), oracle.ACT_SWIGLU)
+    x2 = x.copy()
+    x2[2] *= 37.0
+    y2 = oracle.e4m3_expert(x2, (wg, wu, wd), oracle.ACT_SWIGLU)
+    assert np.array_equal(np.delete(y2, 2, axis=0), np.delete(base, 2, axis=0))
+    wd2 = wd.copy()
+    wd2[5] *= 8.0
+    y3 = oracle.e4m3_expert(x, (wg, wu, wd2), oracle.ACT_SWIGLU)
+    assert np.array_equal(y3[:, 5], 8.0 * base[:, 5])
+    assert np.array_equal(np.delete(y3, 5, axis=1), np.delete(base, 5, axis=1))
+
+
+@pytest.mark.parametrize("act", [0, 1])
+def test_e4m3_expert_stays_close_to_the_float_expert(act):
+    """Each quantised operand is within half an E4M3 step (2^-4 relative) of the
+    float one, so the expert output stays within a few percent of the float
+    expert; a wrong scale (e.g. s instead of 1/s) would be off by orders."""
+    rng = np.random.default_rng(30 + act)
+    x, (wg, wu, wd) = _e4m3_layer_inputs(rng, n=16, d=256, f=128)
+    if act == 0:
+        ref = oracle.swiglu_expert(x, wg, wu, wd)
+        got = oracle.e4m3_expert(x, (wg, wu, wd), act)
+    else:
+        ref = oracle.gelu_expert(x, wu, wd)
+        got = oracle.e4m3_expert(x, (wu, wd), act)
+    err = np.max(np.abs(got - ref)) / np.max(np.abs(ref))
+    assert 1e-4 < err < 0.08

@@ -13,7 +13,8 @@ import pathlib
 __all__ = [
     "MoeError", "MoeConfig", "lib", "make_config", "moe_workspace_bytes", "moe_status_string",
     "moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_forward", "moe_device_status",
-    "moe_permute_noalloc", "moe_expert_capacity", "moe_router_aux_losses",
+    "moe_permute_noalloc", "moe_expert_capacity", "moe_router_aux_losses", "moe_e4m3_weight_bytes",
+    "moe_quantize_e4m3", "MOE_W_NATIVE", "MOE_W_E4M3",
     "MOE_F32", "MOE_BF16", "MOE_SOFTMAX_ALL_RENORM", "MOE_SOFTMAX_TOPK", "MOE_SIGMOID_TOPK_RENORM",
     "MOE_SOFTMAX_ALL_NO_RENORM", "MOE_ACT_SWIGLU", "MOE_ACT_GELU",
     "EXPORTED_SYMBOLS", "LIB_PATH",
@@ -27,11 +28,12 @@ MOE_ERR_BAD_EXPERT_ID = 6
 MOE_F32, MOE_BF16 = 0, 1
 MOE_SOFTMAX_ALL_RENORM, MOE_SOFTMAX_TOPK, MOE_SIGMOID_TOPK_RENORM, MOE_SOFTMAX_ALL_NO_RENORM = 0, 1, 2, 3
 MOE_ACT_SWIGLU, MOE_ACT_GELU = 0, 1
+MOE_W_NATIVE, MOE_W_E4M3 = 0, 1
 
 EXPORTED_SYMBOLS = (
     "moe_workspace_bytes", "moe_status_string", "moe_router_topk", "moe_permute", "moe_grouped_ffn",
     "moe_combine", "moe_forward", "moe_device_status", "moe_permute_noalloc", "moe_expert_capacity",
-    "moe_router_aux_losses",
+    "moe_router_aux_losses", "moe_e4m3_weight_bytes", "moe_quantize_e4m3",
 )
 
 
@@ -56,7 +58,7 @@ class MoeConfig(ctypes.Structure):
         ("expert_act", ctypes.c_int32),
         ("wait_limit_ns", ctypes.c_int64),
         ("capacity_factor", ctypes.c_float),
-        ("reserved", ctypes.c_int32),
+        ("weight_format", ctypes.c_int32),
     ]
 
 
@@ -85,9 +87,12 @@ def lib() -> ctypes.CDLL:
         L.moe_permute_noalloc.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.moe_expert_capacity.argtypes = [cfgp]
         L.moe_router_aux_losses.argtypes = [cfgp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_e4m3_weight_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64]
+        L.moe_quantize_e4m3.argtypes = [vp, ctypes.c_int64, ctypes.c_int32, vp, vp]
         for name in EXPORTED_SYMBOLS[2:]:
             getattr(L, name).restype = i32
         L.moe_expert_capacity.restype = ctypes.c_int64
+        L.moe_e4m3_weight_bytes.restype = sz
         _lib = L
     return _lib
 
@@ -95,9 +100,9 @@ def lib() -> ctypes.CDLL:
 def make_config(T: int, d_model: int, n_experts: int, top_k: int, d_ff: int, dtype: int, gating: int,
                 n_shared: int = 0, d_ff_shared: int = 0, bias_select_only: int = 0,
                 wait_limit_ns: int = 0, expert_act: int = MOE_ACT_SWIGLU,
-                capacity_factor: float = 0.0) -> MoeConfig:
+                capacity_factor: float = 0.0, weight_format: int = MOE_W_NATIVE) -> MoeConfig:
     return MoeConfig(T, d_model, n_experts, top_k, d_ff, n_shared, d_ff_shared, dtype, gating,
-                     bias_select_only, expert_act, wait_limit_ns, capacity_factor, 0)
+                     bias_select_only, expert_act, wait_limit_ns, capacity_factor, weight_format)
 
 
 def _p(v) -> int | None:
@@ -140,6 +145,15 @@ def moe_router_topk(cfg, x, w_router, logit_bias, topk_ids, topk_w, ws, ws_bytes
     nb = ws_bytes if ws_bytes is not None else ws.numel() * ws.element_size()
     _check(lib().moe_router_topk(ctypes.byref(cfg), _p(x), _p(w_router), _p(logit_bias), _p(topk_ids),
                                  _p(topk_w), _p(ws), nb, _stream(stream)), "moe_router_topk")
+
+
+def moe_e4m3_weight_bytes(rows: int, cols: int) -> int:
+    return int(lib().moe_e4m3_weight_bytes(rows, cols))
+
+
+def moe_quantize_e4m3(src, rows: int, cols: int, blob, stream=None) -> None:
+    """bf16 [rows, cols] -> E4M3 blob (codes, then one fp32 scale per row)."""
+    _check(lib().moe_quantize_e4m3(_p(src), rows, cols, _p(blob), _stream(stream)), "moe_quantize_e4m3")
 
 
 def moe_router_aux_losses(cfg, x, w_router, counts, out, ws, ws_bytes=None, stream=None) -> None:

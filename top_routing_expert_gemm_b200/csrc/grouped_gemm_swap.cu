@@ -21,16 +21,18 @@
 //   GEMM-1 (GELU, the two-matrix expert): h^T = GELU(Wu[128 rows] x_perm^T).
 //   GEMM-2 (plain):  y^T[d-block, tokens] = Wd[128 rows] h^T.
 //
-// A unit is (expert, weight-row block j, token chunk of up to BN tokens).
+// A unit is (expert, weight-row block j, token chunk of up to BN tokens; an
+// expert's tokens are cut into chunks of equal size).
 // Inside an expert the units run over blocks of 8 chunks, then j, then the
 // chunk: units running together share weight blocks and token chunks through
 // L2 even for an expert with thousands of tokens.
 //
 // Two schedules (template STREAMK):
-//   * large batches (BN = 256): unit u runs on CTA u mod gridDim (persistent
-//     CTAs, every unit whole);
-//   * decode (BN = 64, STREAMK): the reduction steps of all units, laid end to
-//     end, are cut into one equal contiguous range per CTA, so every CTA
+//   * round robin: unit u runs on CTA u mod gridDim (persistent CTAs, every
+//     unit whole);
+//   * decode (BN = 64, STREAMK, the one the library uses): the reduction steps
+//     of all units, laid end to end, are cut into one equal contiguous range
+//     per CTA, so every CTA
 //     streams the same number of weight bytes whatever the routing.  A unit
 //     cut between CTAs is finished by the last contributor to arrive: each
 //     writes its fp32 partial tile (at most two per CTA: its first and last
@@ -89,6 +91,8 @@ struct SwapParams {
   int64_t counter_cap;     // units the counters (and the schedule) allow
   int* status;
   uint64_t wait_limit_ns;
+  const float* sx;         // FP8: per-token scales of the B operand
+  const float* sw;         // FP8: per-row scales of the weight tensor
 };
 
 template <int BN>
@@ -116,6 +120,7 @@ __device__ __forceinline__ bool epi_bar_any(bool v) {
 
 struct Unit {
   int g, j, chunk;
+  int row0;     // first row of the chunk inside its group
   int n_valid;  // tokens of this chunk (1..BN)
   int nmma;     // MMA N: n_valid rounded up to 16
 };
@@ -137,7 +142,12 @@ __device__ __forceinline__ Unit decode_unit(int64_t u, int J, const int* cum, co
   const int nb = min(S_CB, nch - cb * S_CB);  // chunks in this block
   r.j = (int)(rest / nb);
   r.chunk = cb * S_CB + (int)(rest % nb);
-  r.n_valid = min(bn, off[lo + 1] - off[lo] - r.chunk * bn);
+  // the group's rows split into nch chunks of equal size (a multiple of 16,
+  // at most bn), the last one shorter: no chunk is a sliver next to a full one
+  const int n = off[lo + 1] - off[lo];
+  const int cs = ((n + nch - 1) / nch + 15) & ~15;
+  r.row0 = r.chunk * cs;
+  r.n_valid = min(cs, n - r.row0);
   r.nmma = (r.n_valid + 15) & ~15;
   return r;
 }
@@ -169,7 +179,9 @@ __device__ __forceinline__ void for_each_segment(int64_t n_units, int kb_count, 
   }
 }
 
-template <int EPI, int BN, bool STREAMK>
+// FP8: weights and tokens are E4M3 codes; a stage's 128-byte K slice holds 128
+// of them (kind::f8f6f4) and the epilogue applies the weight-row and token scales.
+template <int EPI, int BN, bool STREAMK, bool FP8>
 __global__ void __launch_bounds__(S_THREADS, 1)
     grouped_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX64,
                              const __grid_constant__ CUtensorMap tmX16, const SwapParams p) {
@@ -248,7 +260,8 @@ __global__ void __launch_bounds__(S_THREADS, 1)
   tc_fence_after();
 
   const uint32_t tmem_base = *tmem_slot;
-  const int kb_count = (p.K + S_BK - 1) / S_BK;
+  constexpr int KB = FP8 ? 2 * S_BK : S_BK;  // elements per 128-byte K slice
+  const int kb_count = (p.K + KB - 1) / KB;
   int64_t n_units = (int64_t)s_cum[G] * p.J;
   if (n_units > p.counter_cap) {  // the host sized the schedule for fewer units: do nothing
     if (threadIdx.x == 0) set_status(p.status, kDevInternal);
@@ -263,7 +276,7 @@ __global__ void __launch_bounds__(S_THREADS, 1)
       for_each_segment<STREAMK>(n_units, kb_count, [&](int64_t u, int kb0, int kb1, bool) {
         const Unit un = decode_unit(u, p.J, s_cum, s_off, G, BN);
         const int w_row = (int)((int64_t)un.g * p.a_group_rows + (int64_t)un.j * (SWIGLU ? S_BM / 2 : S_BM));
-        const int x_row = s_off[un.g] + un.chunk * BN;
+        const int x_row = s_off[un.g] + un.row0;
         const uint32_t tx = S_A_BYTES + (uint32_t)un.nmma * S_BK * 2;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, p.wait_limit_ns, p.status))
@@ -273,15 +286,15 @@ __global__ void __launch_bounds__(S_THREADS, 1)
           fill_par[stage] = (int)phase;
           const uint32_t a_dst = smem_u32(sA + stage * S_A_BYTES);
           if (SWIGLU) {  // 64 gate rows, then the 64 matching up rows
-            tma_load_2d(a_dst, &tmW, fb, kb * S_BK, w_row);
-            tma_load_2d(a_dst + S_A_BYTES / 2, &tmW, fb, kb * S_BK, w_row + p.up_off);
+            tma_load_2d(a_dst, &tmW, fb, kb * KB, w_row);
+            tma_load_2d(a_dst + S_A_BYTES / 2, &tmW, fb, kb * KB, w_row + p.up_off);
           } else {
-            tma_load_2d(a_dst, &tmW, fb, kb * S_BK, w_row);
+            tma_load_2d(a_dst, &tmW, fb, kb * KB, w_row);
           }
           const uint32_t b_dst = smem_u32(sB + stage * B_BYTES);
           int b = 0;
-          for (; b + 64 <= un.nmma; b += 64) tma_load_2d(b_dst + b * S_BK * 2, &tmX64, fb, kb * S_BK, x_row + b);
-          for (; b < un.nmma; b += 16) tma_load_2d(b_dst + b * S_BK * 2, &tmX16, fb, kb * S_BK, x_row + b);
+          for (; b + 64 <= un.nmma; b += 64) tma_load_2d(b_dst + b * 128, &tmX64, fb, kb * KB, x_row + b);
+          for (; b < un.nmma; b += 16) tma_load_2d(b_dst + b * 128, &tmX16, fb, kb * KB, x_row + b);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -299,7 +312,7 @@ __global__ void __launch_bounds__(S_THREADS, 1)
       uint32_t acc_phase = 0;
       for_each_segment<STREAMK>(n_units, kb_count, [&](int64_t u, int kb0, int kb1, bool) {
         const Unit un = decode_unit(u, p.J, s_cum, s_off, G, BN);
-        const uint32_t idesc = idesc_bf16_f32(S_BM, un.nmma);
+        const uint32_t idesc = idesc_f32acc<FP8>(S_BM, un.nmma);
         if (!mbar_wait_bounded(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, p.wait_limit_ns, p.status))
           return false;
         tc_fence_after();
@@ -309,10 +322,7 @@ __global__ void __launch_bounds__(S_THREADS, 1)
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * S_A_BYTES);
           const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
-#pragma unroll
-          for (int kk = 0; kk < S_BK / 16; ++kk)
-            mma_bf16(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32), idesc,
-                     (kb != kb0 || kk != 0) ? 1u : 0u);
+          mma_kslice<FP8>(d_tmem, a0, b0, idesc, kb == kb0);
           mma_commit(smem_u32(&empty[stage]));
           if (++stage == STAGES) {
             stage = 0;
@@ -338,9 +348,16 @@ __global__ void __launch_bounds__(S_THREADS, 1)
     // 16-byte stores.  SwiGLU: a gate row and its up row sit in different
     // warps, so gate rows finish tokens 0..15 and up rows tokens 16..31, each
     // taking the other half's partner values through shared memory.
-    auto finish = [&](const Unit& un, const float (&v)[32], int cc) {
+    auto finish = [&](const Unit& un, float (&v)[32], int cc) {
       const int nv = min(32, un.n_valid - 32 * cc);
-      const int64_t row0 = (int64_t)s_off[un.g] + (int64_t)un.chunk * BN + 32 * cc;
+      const int64_t row0 = (int64_t)s_off[un.g] + un.row0 + 32 * cc;
+      if (FP8) {  // accumulator * weight-row scale * token scale
+        const int feat = SWIGLU ? un.j * 64 + (r & 63) : un.j * S_BM + r;
+        const int64_t wrow = (int64_t)un.g * p.a_group_rows + (SWIGLU && r >= 64 ? p.up_off : 0) + feat;
+        const float sw = feat < p.n_out ? p.sw[wrow] : 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= i < nv ? sw * p.sx[row0 + i] : 0.f;
+      }
       int ncols, col0;
       if (SWIGLU) {
         const int f = r & 63;
@@ -493,10 +510,10 @@ __global__ void __launch_bounds__(S_THREADS, 1)
   }
 }
 
-template <int EPI, int BN, bool STREAMK>
+template <int EPI, int BN, bool STREAMK, bool FP8>
 cudaError_t launch_swap(const CUtensorMap& tw, const CUtensorMap& tx64, const CUtensorMap& tx16,
                         const SwapParams& p, int grid, cudaStream_t stream) {
-  auto kernel = grouped_gemm_swap_kernel<EPI, BN, STREAMK>;
+  auto kernel = grouped_gemm_swap_kernel<EPI, BN, STREAMK, FP8>;
   const size_t smem = swap_smem_bytes<BN>(p.G);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -511,12 +528,15 @@ cudaError_t launch_swap(const CUtensorMap& tw, const CUtensorMap& tx64, const CU
 // Units of one GEMM, bounded from the row count (the chunking is per group).
 int64_t unit_bound(int64_t rows, int G, int bn, int J) { return ((rows + bn - 1) / bn + G) * (int64_t)J; }
 
-// Both GEMMs of the expert FFN with one schedule.
-template <int BN, bool STREAMK>
+// Both GEMMs of the expert FFN with one schedule.  FP8: `a` holds E4M3 codes
+// with per-row scales a.sa, the weights are E4M3 blobs (codes, then per-row
+// scales), and h is re-quantised per token row between the two GEMMs.
+template <int BN, bool STREAMK, bool FP8>
 cudaError_t run_swap(const GroupedFfnArgs& a, cudaStream_t stream) {
   const int G = a.offsets ? a.G : 1;
   const uint64_t lim = a.wait_limit_ns ? a.wait_limit_ns : 2000000000ull;
   const int sms = device_sm_count();
+  const int eb = FP8 ? 1 : 2;
   const bool gelu = a.act == kEpiGELU;
   const int J1 = gelu ? (a.f + 127) / 128 : (a.f + 63) / 64, J2 = (a.d + 127) / 128;
   const int64_t cap1 = unit_bound(a.rows, G, BN, J1), cap2 = unit_bound(a.rows, G, BN, J2);
@@ -528,23 +548,37 @@ cudaError_t run_swap(const GroupedFfnArgs& a, cudaStream_t stream) {
   // GEMM-1: SwiGLU weight blocks of 64 gate + 64 up rows, or GELU blocks of
   // 128 up rows; tokens of x_perm
   const int64_t w1_rows = (gelu ? 1 : 2) * (int64_t)a.f;
+  const float* s1 = FP8 ? reinterpret_cast<const float*>(static_cast<const uint8_t*>(a.w_gate_up) +
+                                                         e4m3_codes_bytes((int64_t)a.G * w1_rows, a.d))
+                        : nullptr;
   CUtensorMap w1, x1a, x1b;
-  if (!make_map(&w1, a.w_gate_up, (uint64_t)a.G * w1_rows, a.d, gelu ? S_BM : 64) ||
-      !make_map(&x1a, a.a, a.rows, a.d, 64) || !make_map(&x1b, a.a, a.rows, a.d, 16))
+  if (!make_map(&w1, a.w_gate_up, (uint64_t)a.G * w1_rows, a.d, gelu ? S_BM : 64, eb) ||
+      !make_map(&x1a, a.a, a.rows, a.d, 64, eb) || !make_map(&x1b, a.a, a.rows, a.d, 16, eb))
     return cudaErrorInvalidValue;
   SwapParams p1{a.offsets, G, a.rows, a.d, a.f, J1, w1_rows, a.f, static_cast<__nv_bfloat16*>(a.h), a.f,
-                a.partial, a.counters, STREAMK ? a.counter_cap : cap1, a.status, lim};
-  cudaError_t e = gelu ? launch_swap<kEpiGELU, BN, STREAMK>(w1, x1a, x1b, p1, grid_for(cap1), stream)
-                       : launch_swap<kEpiSwiGLU, BN, STREAMK>(w1, x1a, x1b, p1, grid_for(cap1), stream);
+                a.partial, a.counters, STREAMK ? a.counter_cap : cap1, a.status, lim, a.sa, s1};
+  cudaError_t e = gelu ? launch_swap<kEpiGELU, BN, STREAMK, FP8>(w1, x1a, x1b, p1, grid_for(cap1), stream)
+                       : launch_swap<kEpiSwiGLU, BN, STREAMK, FP8>(w1, x1a, x1b, p1, grid_for(cap1), stream);
   if (e != cudaSuccess) return e;
+  const void* b2 = a.h;
+  const float* sx2 = nullptr;
+  if (FP8) {  // h -> E4M3 codes and per-token scales
+    e = launch_quantize_e4m3(a.h, a.rows, a.offsets ? a.offsets + a.G : nullptr, a.f, a.hq, a.sh, stream);
+    if (e != cudaSuccess) return e;
+    b2 = a.hq;
+    sx2 = a.sh;
+  }
+  const float* s2 = FP8 ? reinterpret_cast<const float*>(static_cast<const uint8_t*>(a.w_down) +
+                                                         e4m3_codes_bytes((int64_t)a.G * a.d, a.f))
+                        : nullptr;
   // GEMM-2: weight blocks of 128 down rows, tokens of h
   CUtensorMap w2, x2a, x2b;
-  if (!make_map(&w2, a.w_down, (uint64_t)a.G * a.d, a.f, S_BM) || !make_map(&x2a, a.h, a.rows, a.f, 64) ||
-      !make_map(&x2b, a.h, a.rows, a.f, 16))
+  if (!make_map(&w2, a.w_down, (uint64_t)a.G * a.d, a.f, S_BM, eb) || !make_map(&x2a, b2, a.rows, a.f, 64, eb) ||
+      !make_map(&x2b, b2, a.rows, a.f, 16, eb))
     return cudaErrorInvalidValue;
   SwapParams p2{a.offsets, G, a.rows, a.f, a.d, J2, (int64_t)a.d, 0, static_cast<__nv_bfloat16*>(a.y), a.d,
-                a.partial, a.counters, STREAMK ? a.counter_cap : cap2, a.status, lim};
-  return launch_swap<kEpiNone, BN, STREAMK>(w2, x2a, x2b, p2, grid_for(cap2), stream);
+                a.partial, a.counters, STREAMK ? a.counter_cap : cap2, a.status, lim, sx2, s2};
+  return launch_swap<kEpiNone, BN, STREAMK, FP8>(w2, x2a, x2b, p2, grid_for(cap2), stream);
 }
 
 }  // namespace
@@ -568,12 +602,8 @@ cudaError_t launch_grouped_ffn_bf16_decode(const GroupedFfnArgs& a, cudaStream_t
   if (a.rows == 0) return cudaSuccess;
   if (a.partial == nullptr || a.counters == nullptr || a.partial_slots < decode_partial_slots())
     return cudaErrorInvalidValue;
-  return tc::run_swap<kDecodeTokens, true>(a, stream);
+  return a.fp8 ? tc::run_swap<kDecodeTokens, true, true>(a, stream) : tc::run_swap<kDecodeTokens, true, false>(a, stream);
 }
 
-cudaError_t launch_grouped_ffn_bf16_swap(const GroupedFfnArgs& a, cudaStream_t stream) {
-  if (a.rows == 0) return cudaSuccess;
-  return tc::run_swap<256, false>(a, stream);
-}
 
 }  // namespace moe

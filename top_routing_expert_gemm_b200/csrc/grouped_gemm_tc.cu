@@ -56,15 +56,17 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// bf16 row-major [rows, cols] tensor, box = box_rows x 64 columns, 128-byte swizzle
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// row-major [rows, cols] tensor of bf16 or 8-bit elements, box = box_rows x
+// one 128-byte swizzle row (64 bf16 or 128 e4m3)
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows, int elem_bytes) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64u, box_rows};  // 64 bf16 = one 128-byte swizzle row
+  cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
+  cuuint32_t box[2] = {128u / (cuuint32_t)elem_bytes, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -93,6 +95,10 @@ struct Params {
   int* status;
   uint64_t wait_limit_ns;
   int n_mma;               // MMA N (256, or the padded expert count of the router)
+  // 8-bit operands only: per-row scales of A (tokens) and of B (weight rows,
+  // indexed like the rows of the B tensor map)
+  const float* sa;
+  const float* sb;
   // router epilogue only
   const float* bias;       // [E] or null
   int32_t* ids;            // [rows, k]
@@ -121,7 +127,10 @@ __device__ __forceinline__ void decode_tile(int64_t t, int nt, const int* cum, i
 }
 
 
-template <int MODE, int KMAX>
+// FP8: A and B are E4M3 codes; a stage's 128-byte K slice holds 128 of them
+// (kind::f8f6f4, K = 32 per MMA) instead of 64 bf16, and the epilogue scales
+// each accumulator by its token's and its weight row's scale.
+template <int MODE, int KMAX, bool FP8>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const Params p) {
@@ -196,7 +205,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const uint32_t tmem_base = *tmem_slot;
   const int64_t total = (int64_t)s_cum[G] * p.nt;
-  const int kb_count = (p.K + BK - 1) / BK;
+  constexpr int KB = FP8 ? 2 * BK : BK;  // elements per 128-byte K slice
+  const int kb_count = (p.K + KB - 1) / KB;
   const int n_mma = p.n_mma;
   const int bno = MODE == MODE_SWIGLU ? n_mma / 2 : n_mma;  // output columns per tile
 
@@ -219,12 +229,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t fb = smem_u32(&full[stage]);
           mbar_expect_tx(fb, A_BYTES + n_mma * BK * 2);
           fill_par[stage] = (int)phase;
-          tma_load_2d(smem_u32(sA + stage * A_BYTES), &tmA, fb, kb * BK, a_row);
+          tma_load_2d(smem_u32(sA + stage * A_BYTES), &tmA, fb, kb * KB, a_row);
           if (MODE == MODE_SWIGLU) {  // gate rows, then the matching up rows (bno is a multiple of 8)
-            tma_load_2d(smem_u32(sB + stage * B_BYTES), &tmB, fb, kb * BK, b_row);
-            tma_load_2d(smem_u32(sB + stage * B_BYTES + bno * BK * 2), &tmB, fb, kb * BK, b_row + p.up_off);
+            tma_load_2d(smem_u32(sB + stage * B_BYTES), &tmB, fb, kb * KB, b_row);
+            tma_load_2d(smem_u32(sB + stage * B_BYTES + bno * 128), &tmB, fb, kb * KB, b_row + p.up_off);
           } else {
-            tma_load_2d(smem_u32(sB + stage * B_BYTES), &tmB, fb, kb * BK, b_row);
+            tma_load_2d(smem_u32(sB + stage * B_BYTES), &tmB, fb, kb * KB, b_row);
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -237,7 +247,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      const uint32_t idesc = idesc_bf16_f32(BM, n_mma);
+      const uint32_t idesc = idesc_f32acc<FP8>(BM, n_mma);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -255,10 +265,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
           const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            mma_bf16(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32), idesc,
-                     (kb | kk) != 0 ? 1u : 0u);
+          mma_kslice<FP8>(d_tmem, a0, b0, idesc, kb == 0);
           mma_commit(smem_u32(&empty[stage]));
           if (++stage == STAGES) {
             stage = 0;
@@ -291,6 +298,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int col_base = ntile * bno;
       const int col_lim = min(p.N, col_base + bno);  // this tile's columns (bno need not be a multiple of 32)
       __nv_bfloat16* orow = out + grow * p.ldo + col_base;
+      // 8-bit operands: this row's token scale; weight-row scales of the tile's columns
+      const float s_row = FP8 && ok ? p.sa[grow] : 1.f;
+      const float* sg = FP8 ? p.sb + (int64_t)g * p.b_group_rows + col_base : nullptr;
       if (MODE != MODE_ROUTER) {
         // SwiGLU mode: gate in accumulator columns [0, bno), up in [bno, 2 bno);
         // plain mode: the bno output columns
@@ -305,9 +315,20 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               float h0 = __uint_as_float(v[2 * j]), h1 = __uint_as_float(v[2 * j + 1]);
+              float u0 = MODE == MODE_SWIGLU ? __uint_as_float(u[2 * j]) : 0.f;
+              float u1 = MODE == MODE_SWIGLU ? __uint_as_float(u[2 * j + 1]) : 0.f;
+              if (FP8) {  // columns past N read no scale (their outputs are never stored)
+                const int c0 = col_base + c + 2 * j;
+                h0 *= s_row * (c0 < col_lim ? sg[c + 2 * j] : 0.f);
+                h1 *= s_row * (c0 + 1 < col_lim ? sg[c + 2 * j + 1] : 0.f);
+                if (MODE == MODE_SWIGLU) {
+                  u0 *= s_row * (c0 < col_lim ? sg[p.up_off + c + 2 * j] : 0.f);
+                  u1 *= s_row * (c0 + 1 < col_lim ? sg[p.up_off + c + 2 * j + 1] : 0.f);
+                }
+              }
               if (MODE == MODE_SWIGLU) {
-                h0 = silu_f(h0) * __uint_as_float(u[2 * j]);
-                h1 = silu_f(h1) * __uint_as_float(u[2 * j + 1]);
+                h0 = silu_f(h0) * u0;
+                h1 = silu_f(h1) * u1;
               }
               if (MODE == MODE_GELU) {
                 h0 = gelu_f(h0);
@@ -421,55 +442,85 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int MODE, int KMAX>
+template <int MODE, int KMAX, bool FP8 = false>
 cudaError_t launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, int64_t tiles_bound,
                         cudaStream_t stream) {
   const size_t smem = smem_bytes(p.G, MODE == MODE_ROUTER ? p.E : 0);
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<MODE, KMAX>,
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<MODE, KMAX, FP8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int64_t grid = device_sm_count();
   if (tiles_bound < grid) grid = tiles_bound;
   if (grid < 1) grid = 1;
-  grouped_gemm_tc_kernel<MODE, KMAX><<<(unsigned)grid, THREADS, smem, stream>>>(ta, tb, p);
+  grouped_gemm_tc_kernel<MODE, KMAX, FP8><<<(unsigned)grid, THREADS, smem, stream>>>(ta, tb, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 }  // namespace tc
 
-cudaError_t launch_grouped_ffn_bf16_tc(const GroupedFfnArgs& a, cudaStream_t stream) {
-  using namespace tc;
+namespace tc {
+namespace {
+// Both expert GEMMs with token rows as M.  FP8: `a` holds E4M3 codes with
+// per-row scales a.sa, the weights are E4M3 blobs (codes, then per-row
+// scales), and h is re-quantised per token row between the two GEMMs.
+template <bool FP8>
+cudaError_t run_tc(const GroupedFfnArgs& a, cudaStream_t stream) {
   if (a.rows == 0) return cudaSuccess;
   const int G = a.offsets ? a.G : 1;
   const int64_t mt_bound = (a.rows + BM - 1) / BM + (a.offsets ? a.G : 0);
   const uint64_t lim = a.wait_limit_ns ? a.wait_limit_ns : 2000000000ull;
+  const int eb = FP8 ? 1 : 2;
   const int n1 = BN_MMA;
+  const bool gelu = a.act == kEpiGELU;
+  const int64_t w1_rows = (gelu ? 1 : 2) * (int64_t)a.G * a.f;
+  const float* s1 = FP8 ? reinterpret_cast<const float*>(static_cast<const uint8_t*>(a.w_gate_up) +
+                                                         e4m3_codes_bytes(w1_rows, a.d))
+                        : nullptr;
   CUtensorMap mA1, mB1;
   cudaError_t e;
-  if (a.act == kEpiGELU) {
+  if (gelu) {
     // GEMM-1 + GELU: tile = 128 rows x 256 up columns
-    if (!make_map(&mA1, a.a, a.rows, a.d, BM) || !make_map(&mB1, a.w_gate_up, (uint64_t)a.G * a.f, a.d, n1))
+    if (!make_map(&mA1, a.a, a.rows, a.d, BM, eb) || !make_map(&mB1, a.w_gate_up, w1_rows, a.d, n1, eb))
       return cudaErrorInvalidValue;
-    Params p1{a.offsets, G, a.rows, a.d, a.f, (a.f + n1 - 1) / n1, (int64_t)a.f, 0, a.h, a.f, a.status, lim, n1};
-    e = launch_mode<MODE_GELU, 1>(mA1, mB1, p1, mt_bound * p1.nt, stream);
+    Params p1{a.offsets, G, a.rows, a.d, a.f, (a.f + n1 - 1) / n1, (int64_t)a.f, 0, a.h, a.f, a.status, lim, n1,
+              a.sa, s1};
+    e = launch_mode<MODE_GELU, 1, FP8>(mA1, mB1, p1, mt_bound * p1.nt, stream);
   } else {
     // GEMM-1 + SwiGLU: tile = 128 rows x (128 gate + 128 up) columns.  Narrower
     // or non-power-of-two MMA widths measured slower on the layer shapes here.
-    if (!make_map(&mA1, a.a, a.rows, a.d, BM) || !make_map(&mB1, a.w_gate_up, (uint64_t)a.G * 2 * a.f, a.d, n1 / 2))
+    if (!make_map(&mA1, a.a, a.rows, a.d, BM, eb) || !make_map(&mB1, a.w_gate_up, w1_rows, a.d, n1 / 2, eb))
       return cudaErrorInvalidValue;
     Params p1{a.offsets, G, a.rows, a.d, a.f, (a.f + n1 / 2 - 1) / (n1 / 2), 2 * (int64_t)a.f, a.f, a.h, a.f,
-              a.status, lim, n1};
-    e = launch_mode<MODE_SWIGLU, 1>(mA1, mB1, p1, mt_bound * p1.nt, stream);
+              a.status, lim, n1, a.sa, s1};
+    e = launch_mode<MODE_SWIGLU, 1, FP8>(mA1, mB1, p1, mt_bound * p1.nt, stream);
   }
   if (e != cudaSuccess) return e;
+  const void* a2 = a.h;
+  const float* sa2 = nullptr;
+  if (FP8) {  // h -> E4M3 codes and per-token scales
+    e = launch_quantize_e4m3(a.h, a.rows, a.offsets ? a.offsets + a.G : nullptr, a.f, a.hq, a.sh, stream);
+    if (e != cudaSuccess) return e;
+    a2 = a.hq;
+    sa2 = a.sh;
+  }
+  const float* s2 = FP8 ? reinterpret_cast<const float*>(static_cast<const uint8_t*>(a.w_down) +
+                                                         e4m3_codes_bytes((int64_t)a.G * a.d, a.f))
+                        : nullptr;
   // GEMM-2: tile = 128 rows x 256 output columns
   const int n2 = BN_MMA;
   CUtensorMap mA2, mB2;
-  if (!make_map(&mA2, a.h, a.rows, a.f, BM) || !make_map(&mB2, a.w_down, (uint64_t)a.G * a.d, a.f, n2))
+  if (!make_map(&mA2, a2, a.rows, a.f, BM, eb) || !make_map(&mB2, a.w_down, (uint64_t)a.G * a.d, a.f, n2, eb))
     return cudaErrorInvalidValue;
-  Params p2{a.offsets, G, a.rows, a.f, a.d, (a.d + n2 - 1) / n2, (int64_t)a.d, 0, a.y, a.d, a.status, lim, n2};
-  return launch_mode<MODE_PLAIN, 1>(mA2, mB2, p2, mt_bound * p2.nt, stream);
+  Params p2{a.offsets, G, a.rows, a.f, a.d, (a.d + n2 - 1) / n2, (int64_t)a.d, 0, a.y, a.d, a.status, lim, n2,
+            sa2, s2};
+  return launch_mode<MODE_PLAIN, 1, FP8>(mA2, mB2, p2, mt_bound * p2.nt, stream);
+}
+}  // namespace
+}  // namespace tc
+
+cudaError_t launch_grouped_ffn_bf16_tc(const GroupedFfnArgs& a, cudaStream_t stream) {
+  return a.fp8 ? tc::run_tc<true>(a, stream) : tc::run_tc<false>(a, stream);
 }
 
 // Router GEMM on the tensor cores with the top-k and gate weights fused into
@@ -483,7 +534,7 @@ cudaError_t launch_router_topk_tc(const RouterArgs& a, cudaStream_t stream) {
   if (!make_map(&mA, a.x, (uint64_t)a.T, a.d, BM) || !make_map(&mB, a.w_router, (uint64_t)a.E, a.d, n_mma))
     return cudaErrorInvalidValue;
   const uint64_t lim = a.wait_limit_ns ? a.wait_limit_ns : 2000000000ull;
-  Params p{nullptr, 1, a.T, a.d, a.E, 1, 0, 0, nullptr, 0, a.status, lim, n_mma,
+  Params p{nullptr, 1, a.T, a.d, a.E, 1, 0, 0, nullptr, 0, a.status, lim, n_mma, nullptr, nullptr,
            a.bias, a.ids, a.w, a.E, a.k, a.gating, a.bias_select_only};
   const int64_t tiles = (a.T + BM - 1) / BM;
   if (a.k <= 2) return launch_mode<MODE_ROUTER, 2>(mA, mB, p, tiles, stream);

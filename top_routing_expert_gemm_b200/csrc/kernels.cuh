@@ -66,6 +66,13 @@ struct GroupedFfnArgs {
   int act;                // kEpiSwiGLU or kEpiGELU
   int* status;
   uint64_t wait_limit_ns;
+  // 8-bit experts (fp8 set): a holds E4M3 codes with per-row scales sa; the
+  // weights are E4M3 blobs (codes [rows, cols], then fp32 per-row scales at
+  // e4m3_codes_bytes(rows, cols)); hq / sh take h re-quantised per token row
+  bool fp8;
+  const float* sa;
+  uint8_t* hq;
+  float* sh;
   // decode kernel only: fp32 partial tiles of units cut between CTAs, and
   // one arrival counter per unit
   float* partial;
@@ -76,13 +83,18 @@ struct GroupedFfnArgs {
 constexpr int kDecodeMaxCtas = 160;  // CTAs of one decode-schedule launch, at most
 constexpr int kDecodeTokens = 64;    // most tokens per unit of the decode schedule
 cudaError_t launch_grouped_ffn_bf16_tc(const GroupedFfnArgs& a, cudaStream_t stream);      // tcgen05, token rows as M
-cudaError_t launch_grouped_ffn_bf16_swap(const GroupedFfnArgs& a, cudaStream_t stream);    // tcgen05, weight rows as M
-cudaError_t launch_grouped_ffn_bf16_decode(const GroupedFfnArgs& a, cudaStream_t stream);  // the same, split reductions
+cudaError_t launch_grouped_ffn_bf16_decode(const GroupedFfnArgs& a, cudaStream_t stream);  // tcgen05, weight rows as M
 cudaError_t launch_grouped_ffn_f32_simt(const GroupedFfnArgs& a, cudaStream_t stream);      // fp32 CUDA cores
 // decode regime: at most kDecodeTokens rows per touched group on average (uniform-routing expectation)
 bool use_decode_ffn(int64_t rows, int G, bool grouped);
 int64_t decode_partial_slots();  // [128][64] fp32 tiles
 int64_t decode_counter_cap(int64_t rows, int G, int d, int f);
+
+// ---- FP8 E4M3 row quantisation (quant_e4m3.cu): per row s = max|x| / 448,
+// q = e4m3(x / s); rows past *rows_dev (when given) are left alone
+cudaError_t launch_quantize_e4m3(const void* src, int64_t rows, const int32_t* rows_dev, int cols, uint8_t* q,
+                                 float* scale, cudaStream_t stream);
+inline size_t e4m3_codes_bytes(int64_t rows, int64_t cols) { return ((size_t)(rows * cols) + 255) / 256 * 256; }
 
 // ---- combine (combine.cu)
 struct CombineArgs {

@@ -46,7 +46,13 @@ moe_status check_config(const moe_config* c) {
   if (c->expert_act != MOE_ACT_SWIGLU && c->expert_act != MOE_ACT_GELU) return MOE_ERR_INVALID_ARG;
   if (!(c->capacity_factor >= 0.0f) || std::isinf(c->capacity_factor)) return MOE_ERR_INVALID_ARG;
   if (c->bias_select_only != 0 && c->bias_select_only != 1) return MOE_ERR_INVALID_ARG;
-  if (c->reserved != 0 || c->wait_limit_ns < 0) return MOE_ERR_INVALID_ARG;
+  if (c->wait_limit_ns < 0) return MOE_ERR_INVALID_ARG;
+  if (c->weight_format != MOE_W_NATIVE && c->weight_format != MOE_W_E4M3) return MOE_ERR_INVALID_ARG;
+  // 8-bit experts: bf16 activations; rows of 8-bit codes must be whole 16-byte lines
+  if (c->weight_format == MOE_W_E4M3 &&
+      (c->dtype != MOE_BF16 || c->d_model % 16 != 0 || c->d_ff % 16 != 0 ||
+       (c->n_shared > 0 && c->d_ff_shared % 16 != 0)))
+    return MOE_ERR_UNSUPPORTED;
   if (c->n_shared < 0) return MOE_ERR_INVALID_ARG;
   if (c->n_shared > 0 && (c->d_ff_shared <= 0 || c->d_ff_shared % 8 != 0)) return MOE_ERR_INVALID_ARG;
   if (c->n_experts > kMaxExperts || c->top_k > kMaxTopK || c->n_shared > 1) return MOE_ERR_UNSUPPORTED;
@@ -78,6 +84,10 @@ struct Carve {
   int* counters;
   int64_t counter_cap;
   float* aux_part;          // router penalty partial sums [kAuxMaxBlocks][E + 1]
+  // 8-bit experts: E4M3 codes and per-row scales of x_perm, h and the shared
+  // expert's x and h
+  uint8_t *xq, *hq, *xq_s, *hq_s;
+  float *sx, *sh, *sx_s, *sh_s;
   size_t total;
 };
 
@@ -117,6 +127,18 @@ Carve carve(const moe_config* c, void* base) {
     k.y_s = take(eb * c->T * c->d_model);
   }
   k.aux_part = static_cast<float*>(take(sizeof(float) * (size_t)kAuxMaxBlocks * (c->n_experts + 1)));
+  if (c->weight_format == MOE_W_E4M3) {
+    k.xq = static_cast<uint8_t*>(take((size_t)n * c->d_model));
+    k.sx = static_cast<float*>(take(sizeof(float) * n));
+    k.hq = static_cast<uint8_t*>(take((size_t)n * c->d_ff));
+    k.sh = static_cast<float*>(take(sizeof(float) * n));
+    if (c->n_shared > 0) {
+      k.xq_s = static_cast<uint8_t*>(take((size_t)c->T * c->d_model));
+      k.sx_s = static_cast<float*>(take(sizeof(float) * c->T));
+      k.hq_s = static_cast<uint8_t*>(take((size_t)c->T * c->d_ff_shared));
+      k.sh_s = static_cast<float*>(take(sizeof(float) * c->T));
+    }
+  }
   if (decode_routed(c) || decode_shared(c)) {
     k.partial_slots = decode_partial_slots();
     k.partial = static_cast<float*>(take(sizeof(float) * 128 * kDecodeTokens * (size_t)k.partial_slots));
@@ -158,10 +180,22 @@ moe_status bind(const void* p) {
 uint64_t wait_limit(const moe_config* c) { return c->wait_limit_ns > 0 ? (uint64_t)c->wait_limit_ns : 2000000000ull; }
 
 cudaError_t run_ffn(const moe_config* c, const Carve& k, const void* a, const int32_t* offsets, int G, int64_t rows,
-                    int f, const void* w_gu, const void* w_d, void* h, void* y, cudaStream_t s) {
+                    int f, const void* w_gu, const void* w_d, void* h, void* y, cudaStream_t s, bool shared = false) {
   GroupedFfnArgs g{a, offsets, w_gu, w_d, h, y, rows, G, c->d_model, f, c->expert_act, k.status, wait_limit(c),
-                   k.partial, k.partial_slots, k.counters, k.counter_cap};
+                   false, nullptr, nullptr, nullptr, k.partial, k.partial_slots, k.counters, k.counter_cap};
   if (c->dtype != MOE_BF16) return launch_grouped_ffn_f32_simt(g, s);
+  if (c->weight_format == MOE_W_E4M3) {
+    // the expert input -> E4M3 codes and per-token scales (only the rows in use)
+    uint8_t* xq = shared ? k.xq_s : k.xq;
+    float* sx = shared ? k.sx_s : k.sx;
+    const cudaError_t e = launch_quantize_e4m3(a, rows, offsets ? offsets + G : nullptr, c->d_model, xq, sx, s);
+    if (e != cudaSuccess) return e;
+    g.a = xq;
+    g.fp8 = true;
+    g.sa = sx;
+    g.hq = shared ? k.hq_s : k.hq;
+    g.sh = shared ? k.sh_s : k.sh;
+  }
   if (k.partial != nullptr && use_decode_ffn(rows, G, offsets != nullptr)) return launch_grouped_ffn_bf16_decode(g, s);
   return launch_grouped_ffn_bf16_tc(g, s);
 }
@@ -176,6 +210,24 @@ extern "C" {
 size_t moe_workspace_bytes(const moe_config* cfg) {
   if (check_config(cfg) != MOE_OK) return 0;
   return carve(cfg, nullptr).total;
+}
+
+size_t moe_e4m3_weight_bytes(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols <= 0 || cols % 16 != 0) return 0;
+  return e4m3_codes_bytes(rows, cols) + sizeof(float) * (size_t)rows;
+}
+
+moe_status moe_quantize_e4m3(const void* src, int64_t rows, int32_t cols, void* blob, moe_stream_t stream) {
+  if (rows < 0 || cols <= 0 || cols % 16 != 0) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (!src || !blob || !aligned16(src) || (reinterpret_cast<uintptr_t>(blob) % kAlign) != 0)
+    return MOE_ERR_INVALID_ARG;
+  moe_status st;
+  if ((st = bind(blob)) != MOE_OK) return st;
+  uint8_t* q = static_cast<uint8_t*>(blob);
+  float* sc = reinterpret_cast<float*>(q + e4m3_codes_bytes(rows, cols));
+  MOE_CUDA_TRY(launch_quantize_e4m3(src, rows, nullptr, cols, q, sc, stream));
+  return MOE_OK;
 }
 
 int64_t moe_expert_capacity(const moe_config* cfg) {
@@ -318,7 +370,8 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
   MOE_CUDA_TRY(run_ffn(cfg, k, k.x_perm, k.offsets, cfg->n_experts, cfg->T * cfg->top_k, cfg->d_ff, w_gate_up,
                        w_down, k.h, k.y_perm, stream));
   if (cfg->n_shared > 0)
-    MOE_CUDA_TRY(run_ffn(cfg, k, x, nullptr, 1, cfg->T, cfg->d_ff_shared, ws_gate_up, ws_down, k.h_s, k.y_s, stream));
+    MOE_CUDA_TRY(
+        run_ffn(cfg, k, x, nullptr, 1, cfg->T, cfg->d_ff_shared, ws_gate_up, ws_down, k.h_s, k.y_s, stream, true));
   CombineArgs ca{k.y_perm, k.row_of, w, cfg->n_shared > 0 ? k.y_s : nullptr, y, cfg->T, cfg->top_k,
                  cfg->d_model, cfg->dtype == MOE_BF16};
   MOE_CUDA_TRY(launch_combine(ca, stream));

@@ -113,6 +113,16 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[smem] * B[smem]^T for FP8 operands (K = 32 per instruction), fp32 accumulate
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // arrive once on `bar` when every tcgen05 operation issued so far by this thread has completed
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
@@ -144,6 +154,15 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   return d;
 }
 
+// Instruction descriptor of kind::f8f6f4: D fp32, A and B FP8 E4M3 (format 0), both K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4)                        // D format: f32
+         | ((uint32_t)(N >> 3) << 17)     // N / 8
+         | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+template <bool FP8>
+__host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N);
+
 // Instruction descriptor of kind::f16: D fp32, A and B bf16, both K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4)                        // D format: f32
@@ -153,9 +172,29 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | ((uint32_t)(M >> 4) << 24);    // M / 16
 }
 
-// Host: 2-D bf16 row-major [rows, cols] tensor map, box = box_rows x 64
-// columns with the 128-byte swizzle (defined in grouped_gemm_tc.cu).
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+template <>
+__host__ __device__ constexpr uint32_t idesc_f32acc<false>(int M, int N) { return idesc_bf16_f32(M, N); }
+template <>
+__host__ __device__ constexpr uint32_t idesc_f32acc<true>(int M, int N) { return idesc_e4m3_f32(M, N); }
+
+// One 128-byte K slice of a stage: 64 bf16 (4 x K16) or 128 e4m3 (4 x K32);
+// either way the four MMAs start 32 bytes apart inside the swizzled rows.
+template <bool FP8>
+__device__ __forceinline__ void mma_kslice(uint32_t d_tmem, uint32_t a0, uint32_t b0, uint32_t idesc, bool first) {
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    const uint64_t ad = smem_desc_sw128(a0 + kk * 32), bd = smem_desc_sw128(b0 + kk * 32);
+    const uint32_t accum = (!first || kk != 0) ? 1u : 0u;
+    if (FP8) mma_f8(d_tmem, ad, bd, idesc, accum);
+    else mma_bf16(d_tmem, ad, bd, idesc, accum);
+  }
+}
+
+// Host: 2-D row-major [rows, cols] tensor map of bf16 (elem_bytes 2) or 8-bit
+// (elem_bytes 1) elements, box = box_rows x one 128-byte line, 128-byte
+// swizzle (defined in grouped_gemm_tc.cu).
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+              int elem_bytes = 2);
 
 }  // namespace tc
 }  // namespace moe
