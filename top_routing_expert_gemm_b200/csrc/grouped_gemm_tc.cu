@@ -29,7 +29,9 @@
 // Tiles are (group, n-tile, m-tile) with the m-tile fastest, read from the
 // device offsets at kernel start (no host sync): CTAs that run together share
 // one expert's weight panel, so it crosses HBM about once while its row
-// blocks are still in L2.  Rows past a group's end are computed on whatever
+// blocks are still in L2.  An expert with more than 16 m-tiles (a hot expert
+// of skewed routing) is walked in blocks of 16 m-tiles, so its token rows do
+// not fall out of L2 between weight panels.  Rows past a group's end are computed on whatever
 // the TMA box holds (the next group's rows or zero fill) and never stored.
 //
 // Every wait is bounded (Params::wait_limit_ns).  On expiry the CTA raises a
@@ -111,7 +113,13 @@ size_t smem_bytes(int G, int E) {
          sizeof(float) * (size_t)E;
 }
 
-// largest g with cum[g] * nt <= t  (t < cum[G] * nt)
+// m-tiles per block of the tile order: an expert with more m-tiles than this
+// runs them block by block, so its token rows in flight (one block, 2048
+// rows) stay in L2 while every weight panel passes over them
+constexpr int kMBlock = 16;
+
+// tile t -> (group, m-tile, n-tile): group g owns tiles [cum[g]*nt, cum[g+1]*nt);
+// inside it, blocks of kMBlock m-tiles, then the n-tile, then the m-tile
 __device__ __forceinline__ void decode_tile(int64_t t, int nt, const int* cum, int G, int& g, int& mt, int& ntile) {
   int lo = 0, hi = G;
   while (hi - lo > 1) {
@@ -122,8 +130,11 @@ __device__ __forceinline__ void decode_tile(int64_t t, int nt, const int* cum, i
   g = lo;
   const int mtiles = cum[lo + 1] - cum[lo];
   const int64_t local = t - (int64_t)cum[lo] * nt;
-  ntile = (int)(local / mtiles);
-  mt = (int)(local % mtiles);
+  const int mb = (int)(local / ((int64_t)kMBlock * nt));
+  const int64_t rest = local - (int64_t)mb * kMBlock * nt;
+  const int nb = min(kMBlock, mtiles - mb * kMBlock);  // m-tiles in this block
+  ntile = (int)(rest / nb);
+  mt = mb * kMBlock + (int)(rest % nb);
 }
 
 
