@@ -90,6 +90,17 @@ def replica_throughput(tokens_per_rank: int, world: int, ms_max: float) -> float
     return world * tokens_per_rank / (ms_max / 1000.0)
 
 
+def launches_per_step(cfg) -> int:
+    """Kernels of ours one moe_forward step launches: router, dispatch (one
+    block-wide kernel for at most 1024 assignments, else count / scan /
+    scatter) and the row gather, two expert GEMMs per FFN call (routed, and
+    the shared expert's), with 8-bit experts one quantisation before each
+    GEMM, and the combine."""
+    dispatch = 2 if cfg.T * cfg.top_k <= 1024 else 4
+    ffn = 2 + (2 if cfg.e4m3 else 0)
+    return 1 + dispatch + ffn * (1 + cfg.n_shared) + 1
+
+
 def peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -546,7 +557,7 @@ def main() -> None:
         "e2e": {"value": replica_throughput(T, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * d * x_host.element_size(),
                 "d2h_bytes_per_step": T * d * y_host.element_size()},
-        "gpu_launches": args.steps * (8 if cfg.n_shared == 0 else 10),
+        "gpu_launches": args.steps * launches_per_step(cfg),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = {k2: v for k2, v in cpu_baseline(cfg, dev, args.cpu_tokens).items() if k2 != "seconds"}

@@ -18,9 +18,16 @@ def _cuda():
         pytest.skip("no CUDA device")
 
 
-def test_expired_wait_limit_reports_timeout_and_context_survives():
-    # long reductions (d = f = 4096) so that the pipeline's waits outlast a 1 ns limit
-    cfg = synth.LayerConfig("timeout", 1024, 4096, 8, 2, 4096, "bf16", synth.SOFTMAX_TOPK, seed=21)
+@pytest.mark.parametrize("cfg", [
+    # large batch: token-rows-as-M GEMMs; long reductions (d = f = 4096) outlast a 1 ns limit
+    synth.LayerConfig("timeout", 1024, 4096, 8, 2, 4096, "bf16", synth.SOFTMAX_TOPK, seed=21),
+    # decode schedule (split reductions, partial tiles and counters) with the tensor-core router
+    synth.LayerConfig("timeout_decode", 4, 4096, 64, 2, 4096, "bf16", synth.SOFTMAX_TOPK, seed=22),
+    # 8-bit experts with a shared expert
+    synth.LayerConfig("timeout_e4m3", 512, 4096, 8, 2, 2048, "bf16", synth.SOFTMAX_TOPK, n_shared=1,
+                      d_ff_shared=2048, e4m3=True, seed=23),
+], ids=lambda c: c.name)
+def test_expired_wait_limit_reports_timeout_and_context_survives(cfg):
     inp = H.make_inputs(cfg)
     out = H.run_forward(inp, wait_limit_ns=1)
     assert out["status"] == moe.MOE_ERR_TIMEOUT

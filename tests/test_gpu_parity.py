@@ -132,8 +132,9 @@ def test_zero_tokens_is_a_no_op():
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("gating", [0, 1, 2, 3])
 @pytest.mark.parametrize("E,k", [(8, 2), (64, 6), (256, 8)])
-def test_router_topk(dtype, gating, E, k):
-    cfg = synth.LayerConfig("r", 333, 264, E, k, 8, dtype, gating, zipf_s=1.1, bias_select_only=1, seed=E + k)
+@pytest.mark.parametrize("T", [333, 17])  # a warp per token / a block per token (decode-sized batches)
+def test_router_topk(dtype, gating, E, k, T):
+    cfg = synth.LayerConfig("r", T, 264, E, k, 8, dtype, gating, zipf_s=1.1, bias_select_only=1, seed=E + k + T)
     inp = H.make_inputs(cfg)
     c = H.moe_cfg(cfg)
     ws = torch.zeros(moe.moe_workspace_bytes(c), dtype=torch.uint8, device="cuda")

@@ -56,8 +56,13 @@ __device__ __forceinline__ float gelu_f(float z) { return 0.5f * z * (1.0f + erf
 // expert activations (moe_expert_act) and the epilogue of the second GEMM
 constexpr int kEpiSwiGLU = 0, kEpiGELU = 1, kEpiNone = 2;
 
+// A timed-out wait overrides any other code (later kernels of the same call
+// may then read unfinished outputs and report those too); any other code
+// only fills an empty word, so the first failure is the one reported.
 __device__ __forceinline__ void set_status(int* status, int code) {
-  if (status) atomicMax(status, code);
+  if (status == nullptr) return;
+  if (code == kDevTimeout) atomicExch(status, code);
+  else atomicCAS(status, 0, code);
 }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {

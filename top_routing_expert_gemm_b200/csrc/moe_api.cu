@@ -23,9 +23,10 @@ int device_sm_count() {
 // (2*T*d*E flops: 30 GFLOP for T=8192, d=7168, E=256) and runs on the tensor
 // cores with the top-k fused into the epilogue; with few experts (or fp32,
 // which must not use TF32) W_r fits in shared memory and a warp per token on
-// the CUDA cores is cheaper than a 128-token tensor tile.
+// the CUDA cores is cheaper than a 128-token tensor tile; a decode-sized batch
+// (at most 64 tokens) gets a block per token on the CUDA cores either way.
 cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t stream) {
-  if (a.bf16 && a.E >= 64 && a.E <= 256) return launch_router_topk_tc(a, stream);
+  if (a.bf16 && a.E >= 64 && a.E <= 256 && a.T > 64) return launch_router_topk_tc(a, stream);
   return launch_router_topk_simt(a, stream);
 }
 

@@ -145,6 +145,88 @@ __global__ void __launch_bounds__(kThreads) permute_scatter_kernel(const int32_t
   }
 }
 
+// Small dispatch (at most kSmallDispatch assignments, the decode regime): the
+// histogram, the scan and the stable scatter in one block -- a shared-memory
+// histogram, one block scan over the experts, then warp 0 walks the
+// assignments in index order, 32 per round, ranking equal experts with
+// __match_any_sync.  Same results as the three kernels above, two launches
+// fewer.
+constexpr int64_t kSmallDispatch = 1024;
+constexpr int kSmallThreads = 1024;  // >= kMaxExperts: one expert per thread in the scan
+
+__global__ void __launch_bounds__(kSmallThreads)
+    permute_small_kernel(const int32_t* __restrict__ ids, int64_t n, int E, int64_t capacity, int32_t* counts,
+                         int32_t* offsets, int32_t* perm, int32_t* row_of, int* status) {
+  extern __shared__ int sm[];  // hist[E], base[E], run[E]
+  __shared__ int warp_sums[kSmallThreads / 32];
+  int* hist = sm;
+  int* base = sm + E;
+  int* run = sm + 2 * E;
+  const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+  for (int e = tid; e < E; e += kSmallThreads) {
+    hist[e] = 0;
+    run[e] = 0;
+  }
+  __syncthreads();
+  for (int64_t i = tid; i < n; i += kSmallThreads) {
+    const int e = ids[i];
+    if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+    else set_status(status, kDevBadExpertId);
+  }
+  __syncthreads();
+  // exclusive scan of the rows each expert keeps
+  const int total = tid < E ? hist[tid] : 0;
+  const int kept = (int)min((int64_t)total, capacity);
+  int incl = kept;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int v = warp_sums[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, v, off);
+      if (lane >= off) v += u;
+    }
+    warp_sums[lane] = v;
+  }
+  __syncthreads();
+  const int excl = incl - kept + (warp > 0 ? warp_sums[warp - 1] : 0);
+  if (tid < E) {
+    counts[tid] = total;
+    offsets[tid] = excl;
+    base[tid] = excl;
+    if (tid == E - 1) offsets[E] = excl + kept;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const unsigned lt = (1u << lane) - 1u;
+    for (int64_t r0 = 0; r0 < n; r0 += 32) {
+      const int64_t i = r0 + lane;
+      const bool in = i < n;
+      int e = in ? ids[i] : -1;
+      if (e >= E || e < 0) e = -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      int row = -1;
+      if (e >= 0) {
+        const int rank = run[e] + __popc(peers & lt);
+        if (rank < capacity) row = base[e] + rank;
+      }
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(peers) - 1) run[e] += __popc(peers);
+      __syncwarp();
+      if (in) {
+        row_of[i] = row;
+        if (row >= 0) perm[row] = (int32_t)i;
+      }
+    }
+  }
+}
+
 // x_perm[row] = x[perm[row] / k]; one warp per row, 16-byte vectors
 __global__ void __launch_bounds__(kThreads) gather_rows_kernel(const uint8_t* __restrict__ x,
                                                                const int32_t* __restrict__ perm,
@@ -173,12 +255,17 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     return cudaMemsetAsync(a.offsets, 0, sizeof(int32_t) * (a.E + 1), stream);
   }
-  permute_count_kernel<<<n_chunks, kThreads, sizeof(int) * a.E, stream>>>(a.ids, a.n_assign, a.E, a.chunk_counts,
-                                                                          n_chunks, a.status);
-  permute_scan_kernel<<<1, kScanThreads, 0, stream>>>(a.chunk_counts, n_chunks, a.E, a.counts, a.offsets,
-                                                      a.capacity);
-  permute_scatter_kernel<<<n_chunks, kThreads, sizeof(int) * kWarps * a.E, stream>>>(
-      a.ids, a.n_assign, a.E, a.chunk_counts, n_chunks, a.offsets, a.capacity, a.perm, a.row_of);
+  if (a.n_assign <= kSmallDispatch) {
+    permute_small_kernel<<<1, kSmallThreads, 3 * sizeof(int) * a.E, stream>>>(
+        a.ids, a.n_assign, a.E, a.capacity, a.counts, a.offsets, a.perm, a.row_of, a.status);
+  } else {
+    permute_count_kernel<<<n_chunks, kThreads, sizeof(int) * a.E, stream>>>(a.ids, a.n_assign, a.E,
+                                                                            a.chunk_counts, n_chunks, a.status);
+    permute_scan_kernel<<<1, kScanThreads, 0, stream>>>(a.chunk_counts, n_chunks, a.E, a.counts, a.offsets,
+                                                        a.capacity);
+    permute_scatter_kernel<<<n_chunks, kThreads, sizeof(int) * kWarps * a.E, stream>>>(
+        a.ids, a.n_assign, a.E, a.chunk_counts, n_chunks, a.offsets, a.capacity, a.perm, a.row_of);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || a.x == nullptr || a.x_perm == nullptr) return e;
   int64_t blocks = (a.n_assign + kWarps - 1) / kWarps;

@@ -38,6 +38,126 @@ struct RouterParams {
   float* aux_part;  // AUX: [gridDim.x][E + 1] per-block penalty sums
 };
 
+// Top k of kappa = logit + bias over the E logits in shared memory, then the
+// gate weights of the chosen experts; one warp, results for token t.
+template <int KMAX>
+__device__ __forceinline__ void select_and_weigh(const RouterParams& p, const float* logits, int64_t t, int lane) {
+  const int E = p.E, k = p.k;
+  // ---- Keep the top k of kappa = logit + bias
+  TopK<KMAX> tk;
+  tk.init();
+  float mx = -INFINITY;
+  for (int e = lane; e < E; e += 32) {
+    const float kap = logits[e] + (p.bias ? p.bias[e] : 0.f);
+    tk.push(kap, e);
+    mx = fmaxf(mx, kap);
+  }
+  float sel_key[KMAX];
+  int sel_idx[KMAX];
+#pragma unroll
+  for (int s = 0; s < KMAX; ++s) {
+    if (s < k) {
+      float bk = tk.key[0];
+      int bi = tk.idx[0];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        if (ranks_before(ok, oi, bk, bi)) { bk = ok; bi = oi; }
+      }
+      sel_key[s] = bk;
+      sel_idx[s] = bi;
+      if (tk.idx[0] == bi) {  // the owning lane pops its head
+#pragma unroll
+        for (int j = 0; j + 1 < KMAX; ++j) { tk.key[j] = tk.key[j + 1]; tk.idx[j] = tk.idx[j + 1]; }
+        tk.key[KMAX - 1] = -INFINITY;
+        tk.idx[KMAX - 1] = 0x7fffffff;
+      }
+    } else {
+      sel_key[s] = -INFINITY;
+      sel_idx[s] = 0;
+    }
+  }
+
+  // ---- gate weights of the selected experts
+  float wsel[KMAX];
+  float denom = 0.f;
+  if (p.gating == 0 || p.gating == 3) {
+    // softmax over all E, keep the selected probabilities (rule 0 then
+    // renormalises them, rule 3 keeps them as they are)
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    float z = 0.f;
+    for (int e = lane; e < E; e += 32) z += expf(logits[e] + (p.bias ? p.bias[e] : 0.f) - mx);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+#pragma unroll
+    for (int s = 0; s < KMAX; ++s) {
+      wsel[s] = (s < k) ? expf(sel_key[s] - mx) / z : 0.f;
+      denom += wsel[s];
+    }
+  } else if (p.gating == 1) {
+    // softmax over the k kept kappas
+#pragma unroll
+    for (int s = 0; s < KMAX; ++s) {
+      wsel[s] = (s < k) ? expf(sel_key[s] - sel_key[0]) : 0.f;
+      denom += wsel[s];
+    }
+  } else {
+    // sigmoid score, normalised over the selected set
+#pragma unroll
+    for (int s = 0; s < KMAX; ++s) {
+      if (s < k) {
+        const float sc = p.bias_select_only ? logits[sel_idx[s]] : sel_key[s];
+        wsel[s] = 1.0f / (1.0f + expf(-sc));
+      } else {
+        wsel[s] = 0.f;
+      }
+      denom += wsel[s];
+    }
+  }
+#pragma unroll
+  for (int s = 0; s < KMAX; ++s) {
+    if (s < k && lane == s) {
+      p.ids[t * k + s] = sel_idx[s];
+      p.wts[t * k + s] = p.gating == 3 ? wsel[s] : wsel[s] / denom;
+    }
+  }
+}
+
+// Small batches: one block per token; its eight warps split the experts (one
+// full dot product per warp at a time, lanes over d), so a handful of tokens
+// still spreads over many SMs and nothing is staged; warp 0 then selects.
+template <typename T, int KMAX>
+__global__ void __launch_bounds__(kThreads) router_topk_token_block_kernel(RouterParams p) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  float* logits = reinterpret_cast<float*>(smem);  // [E]
+  constexpr int V = Vec16<T>::N;
+  const int d = p.d, E = p.E;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const T* __restrict__ x = static_cast<const T*>(p.x);
+  const T* __restrict__ w = static_cast<const T*>(p.w);
+  for (int64_t t = blockIdx.x; t < p.T; t += gridDim.x) {
+    const T* xr = x + t * d;
+    for (int e = warp; e < E; e += kWarps) {
+      const T* wr = w + (int64_t)e * d;
+      float acc = 0.f;
+#pragma unroll 4
+      for (int i0 = lane * V; i0 < d; i0 += 32 * V) {
+        const Vec16<T> xv = ld16(xr + i0), wv = ld16(wr + i0);
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc = fmaf(Elem<T>::to_f(xv.v[v]), Elem<T>::to_f(wv.v[v]), acc);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (lane == 0) logits[e] = acc;
+    }
+    __syncthreads();
+    if (warp == 0) select_and_weigh<KMAX>(p, logits, t, lane);
+    __syncthreads();
+  }
+}
+
 // Shared memory: logit rows [kWarps][E], with AUX the per-warp penalty sums
 // [kWarps][E] and [kWarps], then W_r [E][d] when staged.
 __host__ __device__ inline size_t router_smem_head(int E, bool aux) {
@@ -133,86 +253,7 @@ __global__ void __launch_bounds__(kThreads) router_topk_simt_kernel(RouterParams
       }
     }
 
-    // ---- Keep the top k of kappa = logit + bias
-    TopK<KMAX> tk;
-    tk.init();
-    float mx = -INFINITY;
-    for (int e = lane; e < E; e += 32) {
-      const float kap = logits[e] + (p.bias ? p.bias[e] : 0.f);
-      tk.push(kap, e);
-      mx = fmaxf(mx, kap);
-    }
-    float sel_key[KMAX];
-    int sel_idx[KMAX];
-#pragma unroll
-    for (int s = 0; s < KMAX; ++s) {
-      if (s < k) {
-        float bk = tk.key[0];
-        int bi = tk.idx[0];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-          if (ranks_before(ok, oi, bk, bi)) { bk = ok; bi = oi; }
-        }
-        sel_key[s] = bk;
-        sel_idx[s] = bi;
-        if (tk.idx[0] == bi) {  // the owning lane pops its head
-#pragma unroll
-          for (int j = 0; j + 1 < KMAX; ++j) { tk.key[j] = tk.key[j + 1]; tk.idx[j] = tk.idx[j + 1]; }
-          tk.key[KMAX - 1] = -INFINITY;
-          tk.idx[KMAX - 1] = 0x7fffffff;
-        }
-      } else {
-        sel_key[s] = -INFINITY;
-        sel_idx[s] = 0;
-      }
-    }
-
-    // ---- gate weights of the selected experts
-    float wsel[KMAX];
-    float denom = 0.f;
-    if (p.gating == 0 || p.gating == 3) {
-      // softmax over all E, keep the selected probabilities (rule 0 then
-      // renormalises them, rule 3 keeps them as they are)
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      float z = 0.f;
-      for (int e = lane; e < E; e += 32) z += expf(logits[e] + (p.bias ? p.bias[e] : 0.f) - mx);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-#pragma unroll
-      for (int s = 0; s < KMAX; ++s) {
-        wsel[s] = (s < k) ? expf(sel_key[s] - mx) / z : 0.f;
-        denom += wsel[s];
-      }
-    } else if (p.gating == 1) {
-      // softmax over the k kept kappas
-#pragma unroll
-      for (int s = 0; s < KMAX; ++s) {
-        wsel[s] = (s < k) ? expf(sel_key[s] - sel_key[0]) : 0.f;
-        denom += wsel[s];
-      }
-    } else {
-      // sigmoid score, normalised over the selected set
-#pragma unroll
-      for (int s = 0; s < KMAX; ++s) {
-        if (s < k) {
-          const float sc = p.bias_select_only ? logits[sel_idx[s]] : sel_key[s];
-          wsel[s] = 1.0f / (1.0f + expf(-sc));
-        } else {
-          wsel[s] = 0.f;
-        }
-        denom += wsel[s];
-      }
-    }
-#pragma unroll
-    for (int s = 0; s < KMAX; ++s) {
-      if (s < k && lane == s) {
-        p.ids[t * k + s] = sel_idx[s];
-        p.wts[t * k + s] = p.gating == 3 ? wsel[s] : wsel[s] / denom;
-      }
-    }
+    select_and_weigh<KMAX>(p, logits, t, lane);
     __syncwarp();
   }
   if (AUX) {  // this block's sums, warps added in a fixed order
@@ -287,9 +328,27 @@ cudaError_t launch_t(const RouterParams& p, int64_t max_blocks, int64_t* blocks_
 // W_r is staged in shared memory when it fits next to the logit rows.
 constexpr size_t kRouterSmemBudget = 160 * 1024;
 
+// Batches up to this many tokens use one block per token.
+constexpr int64_t kTokenBlockMaxT = 64;
+
+template <typename T>
+cudaError_t launch_token_block(const RouterParams& p, cudaStream_t stream) {
+  const size_t smem = sizeof(float) * p.E;
+  auto run = [&](auto kernel) -> cudaError_t {
+    kernel<<<(unsigned)p.T, kThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+  };
+  if (p.k <= 2) return run(router_topk_token_block_kernel<T, 2>);
+  if (p.k <= 4) return run(router_topk_token_block_kernel<T, 4>);
+  if (p.k <= 8) return run(router_topk_token_block_kernel<T, 8>);
+  return run(router_topk_token_block_kernel<T, 16>);
+}
+
 template <bool AUX>
 cudaError_t launch_simt(const RouterArgs& a, int64_t max_blocks, int64_t* blocks, cudaStream_t stream) {
   RouterParams p{a.x, a.w_router, a.bias, a.ids, a.w, a.T, a.d, a.E, a.k, a.gating, a.bias_select_only, a.aux_part};
+  if (!AUX && a.T <= kTokenBlockMaxT)
+    return a.bf16 ? launch_token_block<__nv_bfloat16>(p, stream) : launch_token_block<float>(p, stream);
   const size_t eb = a.bf16 ? 2 : 4;
   const bool fits = router_smem_head(a.E, AUX) + (size_t)a.E * a.d * eb <= kRouterSmemBudget;
   if (a.bf16)
