@@ -53,7 +53,9 @@
  *    T * top_k < 2^31, n_shared in {0, 1}.
  *  - `ws` is caller-owned device scratch of at least moe_workspace_bytes(cfg)
  *    bytes, 256-byte aligned.  Its first 16 bytes hold the device status word
- *    that kernels set on a bounded-wait expiry or an out-of-range expert id;
+ *    that kernels set on a bounded-wait expiry or an out-of-range expert id
+ *    (a bounded-wait expiry overrides any other code; otherwise the first
+ *    code set stays);
  *    moe_forward clears it on entry; a caller chaining the single-stage entry
  *    points zeroes those 16 bytes before the first of them.  moe_device_status()
  *    reads it.

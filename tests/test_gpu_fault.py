@@ -21,8 +21,10 @@ def _cuda():
 @pytest.mark.parametrize("cfg", [
     # large batch: token-rows-as-M GEMMs; long reductions (d = f = 4096) outlast a 1 ns limit
     synth.LayerConfig("timeout", 1024, 4096, 8, 2, 4096, "bf16", synth.SOFTMAX_TOPK, seed=21),
-    # decode schedule (split reductions, partial tiles and counters) with the tensor-core router
+    # decode schedule (split reductions, partial tiles and counters)
     synth.LayerConfig("timeout_decode", 4, 4096, 64, 2, 4096, "bf16", synth.SOFTMAX_TOPK, seed=22),
+    # tensor-core router (64 experts, more than 64 tokens) ahead of the decode schedule
+    synth.LayerConfig("timeout_router_tc", 256, 4096, 64, 2, 2048, "bf16", synth.SOFTMAX_TOPK, seed=24),
     # 8-bit experts with a shared expert
     synth.LayerConfig("timeout_e4m3", 512, 4096, 8, 2, 2048, "bf16", synth.SOFTMAX_TOPK, n_shared=1,
                       d_ff_shared=2048, e4m3=True, seed=23),
