@@ -1,15 +1,14 @@
-// Grouped expert GEMMs on the sm_100a tensor cores with the operands swapped:
-// an expert's weight rows are the MMA's M operand (128 rows) and its tokens
-// the N operand, so the MMA width follows the expert's token count (rounded up
-// to 16) instead of a fixed 128-row token tile.  An expert with 270 tokens
-// costs 256 + 16 MMA columns rather than three 128-row tiles, and an expert
-// with 3 tokens costs 16.
+// Grouped expert GEMMs of the decode regime (a few tokens per expert) on the
+// sm_100a tensor cores, with the operands swapped: an expert's weight rows are
+// the MMA's M operand (128 rows) and its tokens the N operand, so the MMA width
+// follows the expert's token count (rounded up to 16, at most 64 per unit)
+// instead of a fixed 128-row token tile: an expert with 3 tokens costs an MMA
+// of width 16, and the kernel is a stream of the touched experts' weights.
 //
 // "Mixture of Experts: why a model with 671 billion parameters uses only 37",
 // "How data centres handle it" (tokens grouped by expert, all expert
-// multiplies in one launch over a stacked weight matrix) and "Capacity factor:
-// when tokens don't fit" (dropless: every expert gets exactly its rows, no
-// padding to a fixed size); "Mixture of experts: how MoE works and what it
+// multiplies in one launch over a stacked weight matrix); "Mixture of experts:
+// how MoE works and what it
 // costs", "What mixture of experts costs in compute" (decode per-expert
 // batches are small and memory bound).  Expert FFN: "Mixture of Experts
 // Explained: Routers, Active Parameters and VRAM" (a gated feed-forward block
@@ -21,29 +20,27 @@
 //   GEMM-1 (GELU, the two-matrix expert): h^T = GELU(Wu[128 rows] x_perm^T).
 //   GEMM-2 (plain):  y^T[d-block, tokens] = Wd[128 rows] h^T.
 //
-// A unit is (expert, weight-row block j, token chunk of up to BN tokens; an
-// expert's tokens are cut into chunks of equal size).
-// Inside an expert the units run over blocks of 8 chunks, then j, then the
-// chunk: units running together share weight blocks and token chunks through
-// L2 even for an expert with thousands of tokens.
+// A unit is (expert, weight-row block j, token chunk of up to 64 tokens; an
+// expert's tokens are cut into chunks of equal size).  Inside an expert the
+// units run over blocks of 8 chunks, then j, then the chunk, so units running
+// together share weight blocks and token chunks through L2.
 //
-// Two schedules (template STREAMK):
-//   * round robin: unit u runs on CTA u mod gridDim (persistent CTAs, every
-//     unit whole);
-//   * decode (BN = 64, STREAMK, the one the library uses): the reduction steps
-//     of all units, laid end to end, are cut into one equal contiguous range
-//     per CTA, so every CTA
-//     streams the same number of weight bytes whatever the routing.  A unit
-//     cut between CTAs is finished by the last contributor to arrive: each
-//     writes its fp32 partial tile (at most two per CTA: its first and last
-//     unit), adds its step count to the unit's counter, and the one that
-//     completes the count sums the partials in CTA order -- a fixed order, so
-//     results are deterministic -- and runs the epilogue.  Nothing waits on
-//     another CTA.
+// Schedule (stream-K): the reduction steps of all units, laid end to end, are
+// cut into one equal contiguous range per CTA, so every CTA streams the same
+// number of weight bytes whatever the routing.  A unit cut between CTAs is
+// finished by the last contributor to arrive: each writes its fp32 partial
+// tile (at most two per CTA: its first and last unit), adds its step count to
+// the unit's counter, and the one that completes the count sums the partials
+// in CTA order -- a fixed order, so results are deterministic -- and runs the
+// epilogue.  Nothing waits on another CTA.
+//
+// The same kernel with 256-token units and one whole unit per CTA at a time
+// was measured for large batches and ran 1.3-1.7x slower than the
+// token-rows-as-M kernel of grouped_gemm_tc.cu, which large batches use.
 //
 // Persistent, warp-specialised CTA (192 threads): warp 0 TMA producer, warp 1
 // TMEM allocator and single-thread tcgen05.mma issuer, warps 2-5 epilogue;
-// two accumulators of BN columns so the epilogue of one unit overlaps the
+// two accumulators of 64 columns so the epilogue of one unit overlaps the
 // main loop of the next.  Every wait is bounded; on expiry the CTA raises an
 // abort flag and the device status word, drains its own copies and MMAs,
 // frees its tensor memory and returns.
@@ -68,12 +65,10 @@ constexpr int S_CB = 8;                     // token chunks per block in the uni
 constexpr int S_A_BYTES = S_BM * S_BK * 2;  // 16 KiB
 constexpr int kDevInternal = 7;             // status word: internal size check failed
 
-template <int BN>
-struct Shape {
-  static constexpr int STAGES = BN <= 64 ? 8 : 4;
-  static constexpr int B_BYTES = BN * S_BK * 2;
-  static constexpr int TMEM_COLS = 2 * BN;
-};
+constexpr int BN = kDecodeTokens;           // most tokens per unit (MMA N <= 64)
+constexpr int STAGES = 8;
+constexpr int B_BYTES = BN * S_BK * 2;      // 8 KiB
+constexpr int TMEM_COLS = 2 * BN;           // two accumulators
 
 struct SwapParams {
   const int32_t* offsets;  // [G+1] token-row offsets, or null: one group of `rows`
@@ -86,8 +81,8 @@ struct SwapParams {
   int up_off;              // f (SwiGLU)
   __nv_bfloat16* out;      // [rows, n_out]
   int64_t ldo;
-  float* partial;          // STREAMK: [2 * gridDim.x][128][BN] fp32 partial tiles
-  int* counters;           // STREAMK: one per unit; zero on entry, zero on exit
+  float* partial;          // [2 * gridDim.x][128][BN] fp32 partial tiles
+  int* counters;           // one per unit; zero on entry, zero on exit
   int64_t counter_cap;     // units the counters (and the schedule) allow
   int* status;
   uint64_t wait_limit_ns;
@@ -95,10 +90,8 @@ struct SwapParams {
   const float* sw;         // FP8: per-row scales of the weight tensor
 };
 
-template <int BN>
 size_t swap_smem_bytes(int G) {
-  return 1024 + (size_t)Shape<BN>::STAGES * (S_A_BYTES + Shape<BN>::B_BYTES) + S_STAGE_BYTES + 256 +
-         2 * sizeof(int) * (size_t)(G + 1);
+  return 1024 + (size_t)STAGES * (S_A_BYTES + B_BYTES) + S_STAGE_BYTES + 256 + 2 * sizeof(int) * (size_t)(G + 1);
 }
 
 // Named barrier of the four epilogue warps (barrier 1, 128 threads).
@@ -160,33 +153,26 @@ __device__ __forceinline__ int64_t range_owner(int64_t i, int64_t total, int64_t
 }
 
 // Calls f(unit, kb0, kb1, first) for this CTA's segments in order, until f returns false.
-template <bool STREAMK, typename F>
+template <typename F>
 __device__ __forceinline__ void for_each_segment(int64_t n_units, int kb_count, F&& f) {
-  if (STREAMK) {
-    const int64_t total = n_units * kb_count, parts = gridDim.x;
-    const int64_t begin = range_start(blockIdx.x, total, parts), end = range_start(blockIdx.x + 1, total, parts);
-    for (int64_t pos = begin; pos < end;) {
-      const int64_t u = pos / kb_count;
-      const int kb0 = (int)(pos - u * kb_count);
-      const int kb1 = (end - pos < (int64_t)(kb_count - kb0)) ? kb0 + (int)(end - pos) : kb_count;
-      const bool first = pos == begin;
-      pos += kb1 - kb0;
-      if (!f(u, kb0, kb1, first)) return;
-    }
-  } else {
-    for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x)
-      if (!f(u, 0, kb_count, true)) return;
+  const int64_t total = n_units * kb_count, parts = gridDim.x;
+  const int64_t begin = range_start(blockIdx.x, total, parts), end = range_start(blockIdx.x + 1, total, parts);
+  for (int64_t pos = begin; pos < end;) {
+    const int64_t u = pos / kb_count;
+    const int kb0 = (int)(pos - u * kb_count);
+    const int kb1 = (end - pos < (int64_t)(kb_count - kb0)) ? kb0 + (int)(end - pos) : kb_count;
+    const bool first = pos == begin;
+    pos += kb1 - kb0;
+    if (!f(u, kb0, kb1, first)) return;
   }
 }
 
 // FP8: weights and tokens are E4M3 codes; a stage's 128-byte K slice holds 128
 // of them (kind::f8f6f4) and the epilogue applies the weight-row and token scales.
-template <int EPI, int BN, bool STREAMK, bool FP8>
+template <int EPI, bool FP8>
 __global__ void __launch_bounds__(S_THREADS, 1)
     grouped_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX64,
                              const __grid_constant__ CUtensorMap tmX16, const SwapParams p) {
-  constexpr int STAGES = Shape<BN>::STAGES;
-  constexpr int B_BYTES = Shape<BN>::B_BYTES;
   constexpr bool SWIGLU = EPI == kEpiSwiGLU;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -229,7 +215,7 @@ __global__ void __launch_bounds__(S_THREADS, 1)
     tma_prefetch_desc(&tmX16);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), Shape<BN>::TMEM_COLS);
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
   if (p.offsets) {
@@ -273,7 +259,7 @@ __global__ void __launch_bounds__(S_THREADS, 1)
       // ------------------------------------------------ TMA producer
       int stage = 0;
       uint32_t phase = 0;
-      for_each_segment<STREAMK>(n_units, kb_count, [&](int64_t u, int kb0, int kb1, bool) {
+      for_each_segment(n_units, kb_count, [&](int64_t u, int kb0, int kb1, bool) {
         const Unit un = decode_unit(u, p.J, s_cum, s_off, G, BN);
         const int w_row = (int)((int64_t)un.g * p.a_group_rows + (int64_t)un.j * (SWIGLU ? S_BM / 2 : S_BM));
         const int x_row = s_off[un.g] + un.row0;
@@ -310,7 +296,7 @@ __global__ void __launch_bounds__(S_THREADS, 1)
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for_each_segment<STREAMK>(n_units, kb_count, [&](int64_t u, int kb0, int kb1, bool) {
+      for_each_segment(n_units, kb_count, [&](int64_t u, int kb0, int kb1, bool) {
         const Unit un = decode_unit(u, p.J, s_cum, s_off, G, BN);
         const uint32_t idesc = idesc_f32acc<FP8>(S_BM, un.nmma);
         if (!mbar_wait_bounded(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, p.wait_limit_ns, p.status))
@@ -405,7 +391,7 @@ __global__ void __launch_bounds__(S_THREADS, 1)
       epi_bar();  // the staging buffers are free again
     };
 
-    for_each_segment<STREAMK>(n_units, kb_count, [&](int64_t u, int kb0, int kb1, bool first) {
+    for_each_segment(n_units, kb_count, [&](int64_t u, int kb0, int kb1, bool first) {
       const Unit un = decode_unit(u, p.J, s_cum, s_off, G, BN);
       const bool got = mbar_wait_bounded(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.wait_limit_ns, p.status);
       if (epi_bar_any(!got || *abort_flag)) return false;  // every epilogue warp leaves together
@@ -506,21 +492,20 @@ __global__ void __launch_bounds__(S_THREADS, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, Shape<BN>::TMEM_COLS);
+    tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
-template <int EPI, int BN, bool STREAMK, bool FP8>
+template <int EPI, bool FP8>
 cudaError_t launch_swap(const CUtensorMap& tw, const CUtensorMap& tx64, const CUtensorMap& tx16,
                         const SwapParams& p, int grid, cudaStream_t stream) {
-  auto kernel = grouped_gemm_swap_kernel<EPI, BN, STREAMK, FP8>;
-  const size_t smem = swap_smem_bytes<BN>(p.G);
+  auto kernel = grouped_gemm_swap_kernel<EPI, FP8>;
+  const size_t smem = swap_smem_bytes(p.G);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  if (STREAMK) {  // the counters must read zero on entry (a launch that timed out may leave some set)
-    e = cudaMemsetAsync(p.counters, 0, sizeof(int) * (size_t)p.counter_cap, stream);
-    if (e != cudaSuccess) return e;
-  }
+  // the counters must read zero on entry (a launch that timed out may leave some set)
+  e = cudaMemsetAsync(p.counters, 0, sizeof(int) * (size_t)p.counter_cap, stream);
+  if (e != cudaSuccess) return e;
   kernel<<<(unsigned)grid, S_THREADS, smem, stream>>>(tw, tx64, tx16, p);
   return cudaGetLastError();
 }
@@ -531,7 +516,7 @@ int64_t unit_bound(int64_t rows, int G, int bn, int J) { return ((rows + bn - 1)
 // Both GEMMs of the expert FFN with one schedule.  FP8: `a` holds E4M3 codes
 // with per-row scales a.sa, the weights are E4M3 blobs (codes, then per-row
 // scales), and h is re-quantised per token row between the two GEMMs.
-template <int BN, bool STREAMK, bool FP8>
+template <bool FP8>
 cudaError_t run_swap(const GroupedFfnArgs& a, cudaStream_t stream) {
   const int G = a.offsets ? a.G : 1;
   const uint64_t lim = a.wait_limit_ns ? a.wait_limit_ns : 2000000000ull;
@@ -540,11 +525,8 @@ cudaError_t run_swap(const GroupedFfnArgs& a, cudaStream_t stream) {
   const bool gelu = a.act == kEpiGELU;
   const int J1 = gelu ? (a.f + 127) / 128 : (a.f + 63) / 64, J2 = (a.d + 127) / 128;
   const int64_t cap1 = unit_bound(a.rows, G, BN, J1), cap2 = unit_bound(a.rows, G, BN, J2);
-  if (STREAMK && (cap1 > a.counter_cap || cap2 > a.counter_cap)) return cudaErrorInvalidValue;
-  auto grid_for = [&](int64_t cap) -> int {
-    int64_t g = STREAMK ? std::min(sms, kDecodeMaxCtas) : std::min<int64_t>(sms, cap);
-    return (int)std::max<int64_t>(g, 1);
-  };
+  if (cap1 > a.counter_cap || cap2 > a.counter_cap) return cudaErrorInvalidValue;
+  const int grid = std::max(1, std::min(sms, kDecodeMaxCtas));
   // GEMM-1: SwiGLU weight blocks of 64 gate + 64 up rows, or GELU blocks of
   // 128 up rows; tokens of x_perm
   const int64_t w1_rows = (gelu ? 1 : 2) * (int64_t)a.f;
@@ -556,9 +538,9 @@ cudaError_t run_swap(const GroupedFfnArgs& a, cudaStream_t stream) {
       !make_map(&x1a, a.a, a.rows, a.d, 64, eb) || !make_map(&x1b, a.a, a.rows, a.d, 16, eb))
     return cudaErrorInvalidValue;
   SwapParams p1{a.offsets, G, a.rows, a.d, a.f, J1, w1_rows, a.f, static_cast<__nv_bfloat16*>(a.h), a.f,
-                a.partial, a.counters, STREAMK ? a.counter_cap : cap1, a.status, lim, a.sa, s1};
-  cudaError_t e = gelu ? launch_swap<kEpiGELU, BN, STREAMK, FP8>(w1, x1a, x1b, p1, grid_for(cap1), stream)
-                       : launch_swap<kEpiSwiGLU, BN, STREAMK, FP8>(w1, x1a, x1b, p1, grid_for(cap1), stream);
+                a.partial, a.counters, a.counter_cap, a.status, lim, a.sa, s1};
+  cudaError_t e = gelu ? launch_swap<kEpiGELU, FP8>(w1, x1a, x1b, p1, grid, stream)
+                       : launch_swap<kEpiSwiGLU, FP8>(w1, x1a, x1b, p1, grid, stream);
   if (e != cudaSuccess) return e;
   const void* b2 = a.h;
   const float* sx2 = nullptr;
@@ -577,8 +559,8 @@ cudaError_t run_swap(const GroupedFfnArgs& a, cudaStream_t stream) {
       !make_map(&x2b, b2, a.rows, a.f, 16, eb))
     return cudaErrorInvalidValue;
   SwapParams p2{a.offsets, G, a.rows, a.f, a.d, J2, (int64_t)a.d, 0, static_cast<__nv_bfloat16*>(a.y), a.d,
-                a.partial, a.counters, STREAMK ? a.counter_cap : cap2, a.status, lim, sx2, s2};
-  return launch_swap<kEpiNone, BN, STREAMK, FP8>(w2, x2a, x2b, p2, grid_for(cap2), stream);
+                a.partial, a.counters, a.counter_cap, a.status, lim, sx2, s2};
+  return launch_swap<kEpiNone, FP8>(w2, x2a, x2b, p2, grid, stream);
 }
 
 }  // namespace
@@ -602,7 +584,7 @@ cudaError_t launch_grouped_ffn_bf16_decode(const GroupedFfnArgs& a, cudaStream_t
   if (a.rows == 0) return cudaSuccess;
   if (a.partial == nullptr || a.counters == nullptr || a.partial_slots < decode_partial_slots())
     return cudaErrorInvalidValue;
-  return a.fp8 ? tc::run_swap<kDecodeTokens, true, true>(a, stream) : tc::run_swap<kDecodeTokens, true, false>(a, stream);
+  return a.fp8 ? tc::run_swap<true>(a, stream) : tc::run_swap<false>(a, stream);
 }
 
 
