@@ -54,3 +54,28 @@ def test_full_size_repeat_is_bitwise_identical():
     assert torch.equal(a["y"].view(torch.int16), b["y"].view(torch.int16))
     assert torch.equal(a["ids"], b["ids"]) and torch.equal(a["counts"], b["counts"])
     assert np.all(a["counts"].cpu().numpy() >= 0)
+
+
+@pytest.mark.parametrize("name,n_sample", [("gptoss_bf16", 16), ("mixtral_bf16", 24)])
+def test_full_size_layer_with_8bit_experts(name, n_sample):
+    """The full-size layer with E4M3 expert weights, in the launch configuration
+    the benchmark times with --e4m3; sampled tokens against the oracle's own
+    quantisation of the same bf16 values."""
+    cfg = synth.workload(name, e4m3=True)
+    inp = H.make_inputs(cfg)
+    out = H.run_forward(inp)
+    st = H.check_forward(inp, out, n_sample=n_sample)
+    print(name, "e4m3", st)
+    del inp, out
+    torch.cuda.empty_cache()
+
+
+def test_full_size_layer_with_capacity_factor():
+    """Mixtral-shaped layer with a capacity factor of 1.0 under Zipf(1.2)-skewed
+    routing: the hot experts drop their late tokens (first come, first served)."""
+    cfg = synth.workload("mixtral_bf16", zipf_s=1.2, capacity_factor=1.0)
+    inp = H.make_inputs(cfg)
+    out = H.run_forward(inp)
+    st = H.check_forward(inp, out, n_sample=32)
+    assert st["dropped"] > 0
+    print("capacity", st)
