@@ -342,12 +342,15 @@ def test_router_aux_losses(dtype, E, k, d, T):
 
 
 # ------------------------------------------------------------------ 8-bit experts
-def test_quantize_e4m3_matches_the_oracle_bit_for_bit():
+# row lengths: rows shorter than one unrolled step, and unrolled steps with
+# and without a ragged tail of 16-byte vectors
+@pytest.mark.parametrize("cols", [272, 1040, 2880, 4096, 7168, 7184, 14336])
+def test_quantize_e4m3_matches_the_oracle_bit_for_bit(cols):
     """Codes and scales of moe_quantize_e4m3 equal the oracle's per-row E4M3
     quantisation of the same bf16 values (the rounding decisions are taken
     in float32 on both sides): values exactly, scales exactly."""
-    rng = np.random.default_rng(40)
-    rows, cols = 70, 272
+    rng = np.random.default_rng(40 + cols)
+    rows = 70
     w = rng.standard_normal((rows, cols)).astype(np.float32)
     w[3] = 0.0
     w[5] *= 1e-4
@@ -402,3 +405,44 @@ def test_grouped_ffn_e4m3_against_the_oracle(act, sizes, d, f):
     got = H.device_to_host_f64(y)
     assert not np.any(np.isnan(got))
     assert H.rel_err(got, ref) <= H.TOL["bf16"]
+
+
+def _stage_by_stage(inp):
+    """moe_router_topk -> moe_permute (bf16 x_perm) -> moe_grouped_ffn -> moe_combine."""
+    cfg, dev = inp.cfg, inp.dev
+    c = H.moe_cfg(cfg)
+    T, k, E, d = cfg.T, cfg.top_k, cfg.n_experts, cfg.d_model
+    i32 = dict(dtype=torch.int32, device="cuda")
+    ws = torch.empty(max(256, moe.moe_workspace_bytes(c)), dtype=torch.uint8, device="cuda")
+    ids, w = torch.empty(T, k, **i32), torch.empty(T, k, dtype=torch.float32, device="cuda")
+    moe.moe_router_topk(c, dev["x"], dev["w_router"], dev["bias"], ids, w, ws)
+    counts, offsets = torch.empty(E, **i32), torch.empty(E + 1, **i32)
+    perm, row_of = torch.empty(T * k, **i32), torch.empty(T * k, **i32)
+    x_perm = torch.empty(T * k, d, dtype=torch.bfloat16, device="cuda")
+    moe.moe_permute(c, ids, dev["x"], counts, offsets, perm, row_of, x_perm, ws)
+    y_perm = torch.empty(T * k, d, dtype=torch.bfloat16, device="cuda")
+    q = "_q" if cfg.e4m3 else ""
+    moe.moe_grouped_ffn(c, x_perm, offsets, dev["w_gate_up" + q], dev["w_down" + q], y_perm, ws)
+    y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    moe.moe_combine(c, y_perm, row_of, w, None, y)
+    torch.cuda.synchronize()
+    return y
+
+
+@pytest.mark.parametrize("cfg", [
+    SMALL["e4m3_mixtral_like"],                                   # token-rows-as-M GEMMs
+    SMALL["e4m3_decode"],                                         # decode schedule
+    SMALL["e4m3_gelu"],
+    synth.LayerConfig("e4m3_cap", 333, 2880, 16, 4, 640, "bf16", synth.SOFTMAX_TOPK,
+                      zipf_s=1.2, capacity_factor=0.8, e4m3=True, seed=41),  # dropped slots
+], ids=lambda c: c.name)
+def test_forward_e4m3_equals_the_stage_calls(cfg):
+    """With 8-bit experts moe_forward quantises the dispatched rows straight
+    from x (no bf16 copy); the stage-by-stage path quantises the gathered bf16
+    copy inside moe_grouped_ffn.  Same codes, same GEMMs: the outputs are
+    bitwise equal."""
+    inp = H.make_inputs(cfg)
+    out = H.run_forward(inp)
+    assert out["status"] == 0
+    y = _stage_by_stage(inp)
+    assert torch.equal(out["y"].view(torch.int16), y.view(torch.int16))

@@ -76,13 +76,21 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 
 namespace {
 
-constexpr int BM = 128, BK = 64, STAGES = 4, THREADS = 192;
+constexpr int BM = 128, BK = 64, STAGES = 4;
+constexpr int MODE_SWIGLU = 0, MODE_PLAIN = 1, MODE_ROUTER = 2, MODE_GELU = 3;
+
+// warp 0 TMA, warp 1 MMA, then the epilogue warps: four (one per TMEM lane
+// quarter) with bf16 operands; eight (two per quarter, alternate 32-column
+// chunks) with 8-bit ones, whose K loop is half as long per tile, so that the
+// epilogue of a tile still fits under the next tile's main loop, and in the
+// router, whose per-row top-k selection is a serial chain of compares that
+// two threads per row halve
+template <bool FP8, int MODE>
+constexpr int kThreads = (FP8 || MODE == MODE_ROUTER) ? 320 : 192;
 constexpr int BN_MMA = 256;
 constexpr int A_BYTES = BM * BK * 2;       // 16 KiB
 constexpr int B_BYTES = BN_MMA * BK * 2;   // 32 KiB
 constexpr int TMEM_COLS = 2 * BN_MMA;      // two accumulators
-constexpr int MODE_SWIGLU = 0, MODE_PLAIN = 1, MODE_ROUTER = 2, MODE_GELU = 3;
-
 struct Params {
   const int32_t* offsets;  // [G+1] device, or null: one group of `rows` rows
   int G;
@@ -108,9 +116,15 @@ struct Params {
   int E, k, gating, bias_select_only;
 };
 
+// router: the hand-off from the second epilogue warp of a lane quarter to the
+// first: per row up to 16 (key, index, logit) entries, the maximum and the
+// partial softmax denominator, and two mbarriers
+constexpr int kRouterKMax = 16;
+constexpr size_t kRouterXchgBytes = 16 + sizeof(float) * 128 * (3 * kRouterKMax + 2);
+
 size_t smem_bytes(int G, int E) {
   return 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + 256 + 2 * sizeof(int) * (size_t)(G + 1) +
-         sizeof(float) * (size_t)E;
+         sizeof(float) * (size_t)E + (E > 0 ? 8 + kRouterXchgBytes : 0);
 }
 
 // m-tiles per block of the tile order: an expert with more m-tiles than this
@@ -142,7 +156,7 @@ __device__ __forceinline__ void decode_tile(int64_t t, int nt, const int* cum, i
 // (kind::f8f6f4, K = 32 per MMA) instead of 64 bf16, and the epilogue scales
 // each accumulator by its token's and its weight row's scale.
 template <int MODE, int KMAX, bool FP8>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(kThreads<FP8, MODE>, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -161,6 +175,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   int* s_off = fill_par + STAGES;                          // [G+1]
   int* s_cum = s_off + (p.G + 1);                          // [G+1]
   float* s_bias = reinterpret_cast<float*>(s_cum + (p.G + 1));  // [E], router only
+  // router hand-off (after s_bias, 8-byte aligned)
+  uint64_t* xfull = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(s_bias + p.E) + 7) & ~uintptr_t(7));
+  uint64_t* xempty = xfull + 1;
+  float* x_key = reinterpret_cast<float*>(xfull + 2);  // [KMAX][128]
+  int* x_idx = reinterpret_cast<int*>(x_key + KMAX * 128);
+  float* x_val = reinterpret_cast<float*>(x_idx + KMAX * 128);
+  float* x_mx = x_val + KMAX * 128;  // [128]
+  float* x_z = x_mx + 128;           // [128]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int G = p.G;
@@ -173,9 +195,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&tfull[a]), 1);
-      mbar_init(smem_u32(&tempty[a]), 128);
+      mbar_init(smem_u32(&tempty[a]), kThreads<FP8, MODE> - 64);
     }
     mbar_init(smem_u32(drain), 1);
+    if (MODE == MODE_ROUTER) {
+      mbar_init(smem_u32(xfull), 128);
+      mbar_init(smem_u32(xempty), 128);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -186,9 +212,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     tmem_relinquish();
   }
   if (MODE == MODE_ROUTER)
-    for (int e = threadIdx.x; e < p.E; e += THREADS) s_bias[e] = p.bias ? p.bias[e] : 0.f;
+    for (int e = threadIdx.x; e < p.E; e += kThreads<FP8, MODE>) s_bias[e] = p.bias ? p.bias[e] : 0.f;
   if (p.offsets) {
-    for (int g = threadIdx.x; g <= G; g += THREADS) s_off[g] = p.offsets[g];
+    for (int g = threadIdx.x; g <= G; g += kThreads<FP8, MODE>) s_off[g] = p.offsets[g];
   } else if (threadIdx.x == 0) {
     s_off[0] = 0;
     s_off[1] = (int)p.rows;
@@ -290,12 +316,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else {
-    // -------------------------------------------------- epilogue (warps 2..5)
+    // -------------------------------------------------- epilogue (warps 2..)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    constexpr int kPerQuarter = (kThreads<FP8, MODE> - 64) / 128;  // epilogue warps per lane quarter
+    const int part = (warp - 2) >> 2;                         // which of them this warp is
     const int r = q * 32 + lane;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
     int acc = 0;
     uint32_t acc_phase = 0;
+    uint32_t x_phase = 0;  // router hand-off phase
     for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
       int g, mt, ntile;
       decode_tile(t, p.nt, s_cum, G, g, mt, ntile);
@@ -316,7 +345,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // SwiGLU mode: gate in accumulator columns [0, bno), up in [bno, 2 bno);
         // plain mode: the bno output columns
 #pragma unroll 1
-        for (int c = 0; c < bno; c += 32) {
+        for (int c = 32 * part; c < bno; c += 32 * kPerQuarter) {
           uint32_t v[32], u[32];
           tmem_ld32(tb + c, v);
           if (MODE == MODE_SWIGLU) tmem_ld32(tb + bno + c, u);
@@ -363,13 +392,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       } else {
         // Keep the top k of kappa = logit + bias over the E columns of this row,
-        // then the gate weights of the chosen experts.
+        // then the gate weights of the chosen experts.  The two warps of a lane
+        // quarter take alternate 32-column chunks; the second hands its top k,
+        // maximum and partial softmax denominator to the first, which merges.
         TopK<KMAX> tk;
         tk.init();
         float mx = -INFINITY;
         const int E = p.E;
+        const bool all_e = p.gating == 0 || p.gating == 3;  // softmax over all E: needs the denominator
 #pragma unroll 1
-        for (int c = 0; c < p.n_mma; c += 32) {
+        for (int c = 32 * part; c < p.n_mma; c += 32 * kPerQuarter) {
           uint32_t v[32];
           tmem_ld32(tb + c, v);
           tmem_ld_wait();
@@ -383,10 +415,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
           }
         }
-        float z = 0.f;
-        if (p.gating == 0 || p.gating == 3) {  // softmax over all E: needs the full denominator
+        float z = 0.f;  // sum of exp(kappa - mx) over this part's columns
+        if (all_e) {
 #pragma unroll 1
-          for (int c = 0; c < p.n_mma; c += 32) {
+          for (int c = 32 * part; c < p.n_mma; c += 32 * kPerQuarter) {
             uint32_t v[32];
             tmem_ld32(tb + c, v);
             tmem_ld_wait();
@@ -395,28 +427,58 @@ __global__ void __launch_bounds__(THREADS, 1)
               if (c + j < E) z += expf(__uint_as_float(v[j]) + s_bias[c + j] - mx);
           }
         }
-        if (ok) {
-          float wsel[KMAX];
-          float den = 0.f;
+        bool xok = true;
+        if (part == 1) {
+          xok = mbar_wait_bounded(smem_u32(xempty), x_phase ^ 1u, abort_flag, p.wait_limit_ns, p.status);
+          if (xok) {
 #pragma unroll
-          for (int s = 0; s < KMAX; ++s) {
-            float wv = 0.f;
-            if (s < p.k) {
-              if (p.gating == 0 || p.gating == 3) wv = expf(tk.key[s] - mx) / z;
-              else if (p.gating == 1) wv = expf(tk.key[s] - tk.key[0]);
-              else wv = 1.0f / (1.0f + expf(-(p.bias_select_only ? tk.val[s] : tk.key[s])));
+            for (int s = 0; s < KMAX; ++s) {
+              x_key[s * 128 + r] = tk.key[s];
+              x_idx[s * 128 + r] = tk.idx[s];
+              x_val[s * 128 + r] = tk.val[s];
             }
-            wsel[s] = wv;
-            den += wv;
+            x_mx[r] = mx;
+            x_z[r] = z;
+            mbar_arrive(smem_u32(xfull));
           }
+        } else {
+          xok = mbar_wait_bounded(smem_u32(xfull), x_phase, abort_flag, p.wait_limit_ns, p.status);
+          if (xok) {
 #pragma unroll
-          for (int s = 0; s < KMAX; ++s) {
-            if (s < p.k) {
-              p.ids[grow * p.k + s] = tk.idx[s];
-              p.wts[grow * p.k + s] = p.gating == 3 ? wsel[s] : wsel[s] / den;  // rule 3: not renormalised
+            for (int s = 0; s < KMAX; ++s) tk.push(x_key[s * 128 + r], x_idx[s * 128 + r], x_val[s * 128 + r]);
+            const float mx1 = x_mx[r], z1 = x_z[r];
+            mbar_arrive(smem_u32(xempty));
+            if (all_e) {  // the two partial denominators, brought to the common maximum
+              const float m = fmaxf(mx, mx1);
+              z = z * expf(mx - m) + (z1 > 0.f ? z1 * expf(mx1 - m) : 0.f);
+              mx = m;
+            }
+            if (ok) {
+              float wsel[KMAX];
+              float den = 0.f;
+#pragma unroll
+              for (int s = 0; s < KMAX; ++s) {
+                float wv = 0.f;
+                if (s < p.k) {
+                  if (all_e) wv = expf(tk.key[s] - mx) / z;
+                  else if (p.gating == 1) wv = expf(tk.key[s] - tk.key[0]);
+                  else wv = 1.0f / (1.0f + expf(-(p.bias_select_only ? tk.val[s] : tk.key[s])));
+                }
+                wsel[s] = wv;
+                den += wv;
+              }
+#pragma unroll
+              for (int s = 0; s < KMAX; ++s) {
+                if (s < p.k) {
+                  p.ids[grow * p.k + s] = tk.idx[s];
+                  p.wts[grow * p.k + s] = p.gating == 3 ? wsel[s] : wsel[s] / den;  // rule 3: not renormalised
+                }
+              }
             }
           }
         }
+        x_phase ^= 1u;
+        if (!xok) break;
       }
       tc_fence_before();
       mbar_arrive(smem_u32(&tempty[acc]));
@@ -463,7 +525,7 @@ cudaError_t launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const Para
   int64_t grid = device_sm_count();
   if (tiles_bound < grid) grid = tiles_bound;
   if (grid < 1) grid = 1;
-  grouped_gemm_tc_kernel<MODE, KMAX, FP8><<<(unsigned)grid, THREADS, smem, stream>>>(ta, tb, p);
+  grouped_gemm_tc_kernel<MODE, KMAX, FP8><<<(unsigned)grid, kThreads<FP8, MODE>, smem, stream>>>(ta, tb, p);
   return cudaGetLastError();
 }
 

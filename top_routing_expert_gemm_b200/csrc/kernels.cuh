@@ -94,6 +94,10 @@ int64_t decode_counter_cap(int64_t rows, int G, int d, int f);
 // q = e4m3(x / s); rows past *rows_dev (when given) are left alone
 cudaError_t launch_quantize_e4m3(const void* src, int64_t rows, const int32_t* rows_dev, int cols, uint8_t* q,
                                  float* scale, cudaStream_t stream);
+// the same for dispatched rows: output row r quantises x row perm[r] / k
+cudaError_t launch_gather_quantize_e4m3(const void* x, const int32_t* perm, int k, int64_t rows,
+                                        const int32_t* rows_dev, int cols, uint8_t* q, float* scale,
+                                        cudaStream_t stream);
 inline size_t e4m3_codes_bytes(int64_t rows, int64_t cols) { return ((size_t)(rows * cols) + 255) / 256 * 256; }
 
 // ---- combine (combine.cu)

@@ -120,7 +120,8 @@ Carve carve(const moe_config* c, void* base) {
   k.perm = static_cast<int32_t*>(take(sizeof(int32_t) * n));
   k.row_of = static_cast<int32_t*>(take(sizeof(int32_t) * n));
   k.chunk_counts = static_cast<int32_t*>(take(sizeof(int32_t) * (size_t)c->n_experts * permute_n_chunks(n)));
-  k.x_perm = take(eb * n * c->d_model);
+  // with 8-bit experts moe_forward gathers E4M3 codes (xq) and no bf16 copy
+  k.x_perm = take(c->weight_format == MOE_W_E4M3 ? 0 : eb * n * c->d_model);
   k.h = take(eb * n * c->d_ff);
   k.y_perm = take(eb * n * c->d_model);
   if (c->n_shared > 0) {
@@ -180,8 +181,10 @@ moe_status bind(const void* p) {
 
 uint64_t wait_limit(const moe_config* c) { return c->wait_limit_ns > 0 ? (uint64_t)c->wait_limit_ns : 2000000000ull; }
 
+// a_quantized: 8-bit experts whose input rows are already in xq / sx
 cudaError_t run_ffn(const moe_config* c, const Carve& k, const void* a, const int32_t* offsets, int G, int64_t rows,
-                    int f, const void* w_gu, const void* w_d, void* h, void* y, cudaStream_t s, bool shared = false) {
+                    int f, const void* w_gu, const void* w_d, void* h, void* y, cudaStream_t s, bool shared = false,
+                    bool a_quantized = false) {
   GroupedFfnArgs g{a, offsets, w_gu, w_d, h, y, rows, G, c->d_model, f, c->expert_act, k.status, wait_limit(c),
                    false, nullptr, nullptr, nullptr, k.partial, k.partial_slots, k.counters, k.counter_cap};
   if (c->dtype != MOE_BF16) return launch_grouped_ffn_f32_simt(g, s);
@@ -189,8 +192,10 @@ cudaError_t run_ffn(const moe_config* c, const Carve& k, const void* a, const in
     // the expert input -> E4M3 codes and per-token scales (only the rows in use)
     uint8_t* xq = shared ? k.xq_s : k.xq;
     float* sx = shared ? k.sx_s : k.sx;
-    const cudaError_t e = launch_quantize_e4m3(a, rows, offsets ? offsets + G : nullptr, c->d_model, xq, sx, s);
-    if (e != cudaSuccess) return e;
+    if (!a_quantized) {
+      const cudaError_t e = launch_quantize_e4m3(a, rows, offsets ? offsets + G : nullptr, c->d_model, xq, sx, s);
+      if (e != cudaSuccess) return e;
+    }
     g.a = xq;
     g.fp8 = true;
     g.sa = sx;
@@ -365,11 +370,18 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
   RouterArgs ra{x, w_router, logit_bias, ids, w, cfg->T, cfg->d_model, cfg->n_experts, cfg->top_k,
                 cfg->gating, cfg->bias_select_only, cfg->dtype == MOE_BF16, k.status, wait_limit(cfg)};
   MOE_CUDA_TRY(launch_router_topk(ra, stream));
-  PermuteArgs pa{ids, x, counts, k.offsets, k.perm, k.row_of, k.x_perm, k.chunk_counts, cfg->T * cfg->top_k,
-                 cfg->top_k, cfg->d_model, cfg->n_experts, (int)elem_bytes(cfg), k.status, capacity_rows(cfg)};
+  // 8-bit experts: the dispatch writes no bf16 copy; the expert input rows are
+  // quantised straight from x, gathered by perm
+  const bool e4m3 = cfg->weight_format == MOE_W_E4M3;
+  PermuteArgs pa{ids, x, counts, k.offsets, k.perm, k.row_of, e4m3 ? nullptr : k.x_perm, k.chunk_counts,
+                 cfg->T * cfg->top_k, cfg->top_k, cfg->d_model, cfg->n_experts, (int)elem_bytes(cfg), k.status,
+                 capacity_rows(cfg)};
   MOE_CUDA_TRY(launch_permute(pa, stream));
+  if (e4m3)
+    MOE_CUDA_TRY(launch_gather_quantize_e4m3(x, k.perm, cfg->top_k, cfg->T * cfg->top_k, k.offsets + cfg->n_experts,
+                                             cfg->d_model, k.xq, k.sx, stream));
   MOE_CUDA_TRY(run_ffn(cfg, k, k.x_perm, k.offsets, cfg->n_experts, cfg->T * cfg->top_k, cfg->d_ff, w_gate_up,
-                       w_down, k.h, k.y_perm, stream));
+                       w_down, k.h, k.y_perm, stream, false, e4m3));
   if (cfg->n_shared > 0)
     MOE_CUDA_TRY(
         run_ffn(cfg, k, x, nullptr, 1, cfg->T, cfg->d_ff_shared, ws_gate_up, ws_down, k.h_s, k.y_s, stream, true));

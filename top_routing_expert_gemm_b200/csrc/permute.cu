@@ -239,7 +239,15 @@ __global__ void __launch_bounds__(kThreads) gather_rows_kernel(const uint8_t* __
     const int64_t t = perm[row] / k;
     const uint4* src = reinterpret_cast<const uint4*>(x + t * row_bytes);
     uint4* dst = reinterpret_cast<uint4*>(x_perm + row * row_bytes);
-    for (int64_t j = lane; j < n16; j += 32) dst[j] = __ldg(src + j);
+    int64_t j = lane;
+    for (; j + 96 < n16; j += 128) {  // four independent 16-byte loads in flight per lane
+      const uint4 a0 = __ldg(src + j), a1 = __ldg(src + j + 32), a2 = __ldg(src + j + 64), a3 = __ldg(src + j + 96);
+      dst[j] = a0;
+      dst[j + 32] = a1;
+      dst[j + 64] = a2;
+      dst[j + 96] = a3;
+    }
+    for (; j < n16; j += 32) dst[j] = __ldg(src + j);
   }
 }
 
