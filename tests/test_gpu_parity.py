@@ -148,6 +148,31 @@ def test_router_topk(dtype, gating, E, k, T):
     H.check_routing(cfg, ids.cpu().numpy().astype(np.int64), w.cpu().numpy().astype(np.float64), r, cfg.T)
 
 
+
+# The tensor-core router at model-like widths (d = 1024, 2048), ragged last
+# tile; repeated calls agree bitwise.
+@pytest.mark.parametrize("gating", [0, 1, 2, 3])
+@pytest.mark.parametrize("E,k", [(64, 6), (256, 8), (144, 16)])
+@pytest.mark.parametrize("T,d", [(333, 1024), (1000, 2048)])
+def test_router_topk_long_rows(gating, E, k, T, d):
+    cfg = synth.LayerConfig("rs", T, d, E, k, 8, "bf16", gating, zipf_s=1.1, bias_select_only=1, seed=E + d + T)
+    inp = H.make_inputs(cfg)
+    c = H.moe_cfg(cfg)
+    ws = torch.zeros(moe.moe_workspace_bytes(c), dtype=torch.uint8, device="cuda")
+    out = []
+    for _ in range(2):
+        ids = torch.empty(cfg.T, k, dtype=torch.int32, device="cuda")
+        w = torch.empty(cfg.T, k, dtype=torch.float32, device="cuda")
+        moe.moe_router_topk(c, inp.dev["x"], inp.dev["w_router"], inp.dev["bias"], ids, w, ws)
+        torch.cuda.synchronize()
+        out.append((ids, w))
+    assert torch.equal(out[0][0], out[1][0]) and torch.equal(out[0][1], out[1][1])
+    x = synth.host_tensor(cfg, "x").reshape(cfg.T, cfg.d_model)
+    wr = synth.host_tensor(cfg, "w_router").reshape(E, cfg.d_model)
+    r = oracle.route(x, wr, inp.bias.astype(np.float64), k, gating, cfg.bias_select_only)
+    ids, w = out[0]
+    H.check_routing(cfg, ids.cpu().numpy().astype(np.int64), w.cpu().numpy().astype(np.float64), r, cfg.T)
+
 @pytest.mark.parametrize("T,E,k", [(1, 1, 1), (1000, 8, 2), (4099, 256, 8), (2048, 1024, 16), (333, 5, 5)])
 @pytest.mark.parametrize("skew", ["uniform", "one_expert", "half_empty"])
 @pytest.mark.parametrize("cf", [0.0, 1.0, 0.3])

@@ -116,15 +116,15 @@ struct Params {
   int E, k, gating, bias_select_only;
 };
 
-// router: the hand-off from the second epilogue warp of a lane quarter to the
-// first: per row up to 16 (key, index, logit) entries, the maximum and the
-// partial softmax denominator, and two mbarriers
-constexpr int kRouterKMax = 16;
-constexpr size_t kRouterXchgBytes = 16 + sizeof(float) * 128 * (3 * kRouterKMax + 2);
+// router: the tile's logits are staged in shared memory over the drained
+// operand ring, 260 floats per row (16-byte rows that start on different banks)
+constexpr int kLogStride = 260;
+static_assert(128 * kLogStride * 4 <= STAGES * (A_BYTES + B_BYTES), "router logits fit over the ring");
+constexpr size_t kRouterBarBytes = 8;  // one mbarrier
 
 size_t smem_bytes(int G, int E) {
   return 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + 256 + 2 * sizeof(int) * (size_t)(G + 1) +
-         sizeof(float) * (size_t)E + (E > 0 ? 8 + kRouterXchgBytes : 0);
+         sizeof(float) * (size_t)E + (E > 0 ? 8 + kRouterBarBytes : 0);
 }
 
 // m-tiles per block of the tile order: an expert with more m-tiles than this
@@ -176,13 +176,8 @@ __global__ void __launch_bounds__(kThreads<FP8, MODE>, 1)
   int* s_cum = s_off + (p.G + 1);                          // [G+1]
   float* s_bias = reinterpret_cast<float*>(s_cum + (p.G + 1));  // [E], router only
   // router hand-off (after s_bias, 8-byte aligned)
-  uint64_t* xfull = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(s_bias + p.E) + 7) & ~uintptr_t(7));
-  uint64_t* xempty = xfull + 1;
-  float* x_key = reinterpret_cast<float*>(xfull + 2);  // [KMAX][128]
-  int* x_idx = reinterpret_cast<int*>(x_key + KMAX * 128);
-  float* x_val = reinterpret_cast<float*>(x_idx + KMAX * 128);
-  float* x_mx = x_val + KMAX * 128;  // [128]
-  float* x_z = x_mx + 128;           // [128]
+  uint64_t* lrdy = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(s_bias + p.E) + 7) & ~uintptr_t(7));
+  float* s_log = reinterpret_cast<float*>(smem);  // router: [128][kLogStride] logits over the ring
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int G = p.G;
@@ -199,8 +194,7 @@ __global__ void __launch_bounds__(kThreads<FP8, MODE>, 1)
     }
     mbar_init(smem_u32(drain), 1);
     if (MODE == MODE_ROUTER) {
-      mbar_init(smem_u32(xfull), 128);
-      mbar_init(smem_u32(xempty), 128);
+      mbar_init(smem_u32(lrdy), kThreads<FP8, MODE> - 64);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -324,7 +318,7 @@ __global__ void __launch_bounds__(kThreads<FP8, MODE>, 1)
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
     int acc = 0;
     uint32_t acc_phase = 0;
-    uint32_t x_phase = 0;  // router hand-off phase
+    uint32_t l_phase = 0;  // router: logits staged
     for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
       int g, mt, ntile;
       decode_tile(t, p.nt, s_cum, G, g, mt, ntile);
@@ -391,94 +385,141 @@ __global__ void __launch_bounds__(kThreads<FP8, MODE>, 1)
           }
         }
       } else {
-        // Keep the top k of kappa = logit + bias over the E columns of this row,
-        // then the gate weights of the chosen experts.  The two warps of a lane
-        // quarter take alternate 32-column chunks; the second hands its top k,
-        // maximum and partial softmax denominator to the first, which merges.
-        TopK<KMAX> tk;
-        tk.init();
-        float mx = -INFINITY;
-        const int E = p.E;
-        const bool all_e = p.gating == 0 || p.gating == 3;  // softmax over all E: needs the denominator
+        // Router: keep the top k of kappa = logit + bias over the E columns of
+        // each row, then the gate weights of the chosen experts.  The CTA owns
+        // this one tile (the router launch has a CTA per tile), so its operand
+        // ring is drained: each thread stages its row's logits there (the two
+        // warps of a lane quarter alternate 32-column chunks), then each warp
+        // selects for 16 rows, four at a time (independent chains of shuffles
+        // that the scheduler interleaves): lane l holds columns l, l+32, ...,
+        // and k rounds of a warp-wide (kappa desc, index asc) maximum pick the
+        // experts in order.
 #pragma unroll 1
         for (int c = 32 * part; c < p.n_mma; c += 32 * kPerQuarter) {
           uint32_t v[32];
           tmem_ld32(tb + c, v);
           tmem_ld_wait();
+          float4* dst = reinterpret_cast<float4*>(s_log + r * kLogStride + c);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if (c + j < E) {
-              const float l = __uint_as_float(v[j]);
-              const float kap = l + s_bias[c + j];
-              tk.push(kap, c + j, l);
-              mx = fmaxf(mx, kap);
-            }
-          }
+          for (int j = 0; j < 8; ++j)  // n_mma is a multiple of 16
+            if (c + 4 * j < p.n_mma)
+              dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                   __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
         }
-        float z = 0.f;  // sum of exp(kappa - mx) over this part's columns
-        if (all_e) {
+        mbar_arrive(smem_u32(lrdy));
+        const bool lok = mbar_wait_bounded(smem_u32(lrdy), l_phase, abort_flag, p.wait_limit_ns, p.status);
+        l_phase ^= 1u;
+        if (!lok) break;
+        constexpr int R = 4;                       // rows in flight per warp
+        constexpr int kEpiWarps = kThreads<FP8, MODE> / 32 - 2;
+        const int E = p.E, k = p.k;
+        const bool all_e = p.gating == 0 || p.gating == 3;  // softmax over all E: needs the denominator
+        const int64_t row0 = (int64_t)s_off[g] + (int64_t)mt * BM;
 #pragma unroll 1
-          for (int c = 32 * part; c < p.n_mma; c += 32 * kPerQuarter) {
-            uint32_t v[32];
-            tmem_ld32(tb + c, v);
-            tmem_ld_wait();
+        for (int rb = (warp - 2) * R; rb < BM; rb += kEpiWarps * R) {
+          float key[R][8], lg[R][8], mx[R], z[R], key0[R], sel_key[R], sel_val[R];
+          int sel_idx[R];
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (c + j < E) z += expf(__uint_as_float(v[j]) + s_bias[c + j] - mx);
+          for (int q2 = 0; q2 < R; ++q2) {
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+              const int c = lane + 32 * m;
+              lg[q2][m] = c < E ? s_log[(rb + q2) * kLogStride + c] : 0.f;
+              key[q2][m] = c < E ? lg[q2][m] + s_bias[c] : -INFINITY;
+            }
+            mx[q2] = key[q2][0];
+#pragma unroll
+            for (int m = 1; m < 8; ++m) mx[q2] = fmaxf(mx[q2], key[q2][m]);
+            z[q2] = 0.f;
+            key0[q2] = sel_key[q2] = sel_val[q2] = 0.f;
+            sel_idx[q2] = 0;
+          }
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+            for (int q2 = 0; q2 < R; ++q2) mx[q2] = fmaxf(mx[q2], __shfl_xor_sync(0xffffffffu, mx[q2], off));
+          if (all_e) {
+#pragma unroll
+            for (int q2 = 0; q2 < R; ++q2)
+#pragma unroll
+              for (int m = 0; m < 8; ++m)
+                if (lane + 32 * m < E) z[q2] += expf(key[q2][m] - mx[q2]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+              for (int q2 = 0; q2 < R; ++q2) z[q2] += __shfl_xor_sync(0xffffffffu, z[q2], off);
+          }
+#pragma unroll 1
+          for (int s = 0; s < k; ++s) {
+            float bk[R];
+            int bi[R];
+#pragma unroll
+            for (int q2 = 0; q2 < R; ++q2) {
+              bk[q2] = key[q2][0];
+              bi[q2] = lane;
+#pragma unroll
+              for (int m = 1; m < 8; ++m)
+                if (ranks_before(key[q2][m], lane + 32 * m, bk[q2], bi[q2])) {
+                  bk[q2] = key[q2][m];
+                  bi[q2] = lane + 32 * m;
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+              for (int q2 = 0; q2 < R; ++q2) {
+                const float ok2 = __shfl_xor_sync(0xffffffffu, bk[q2], off);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi[q2], off);
+                if (ranks_before(ok2, oi, bk[q2], bi[q2])) {
+                  bk[q2] = ok2;
+                  bi[q2] = oi;
+                }
+              }
+            }
+#pragma unroll
+            for (int q2 = 0; q2 < R; ++q2) {
+              // the owner lane of the winner takes it out and hands over its raw logit
+              const int owner = bi[q2] & 31, mw = bi[q2] >> 5;
+              float cand = 0.f;
+#pragma unroll
+              for (int m = 0; m < 8; ++m) cand = m == mw ? lg[q2][m] : cand;
+              const float bv = __shfl_sync(0xffffffffu, cand, owner);
+              if (lane == owner) {
+#pragma unroll
+                for (int m = 0; m < 8; ++m) key[q2][m] = m == mw ? -INFINITY : key[q2][m];
+              }
+              if (s == 0) key0[q2] = bk[q2];
+              if (lane == s) {
+                sel_key[q2] = bk[q2];
+                sel_idx[q2] = bi[q2];
+                sel_val[q2] = bv;
+              }
+            }
+          }
+          float wv[R], den[R];
+#pragma unroll
+          for (int q2 = 0; q2 < R; ++q2) {
+            wv[q2] = 0.f;
+            if (lane < k) {
+              if (all_e) wv[q2] = expf(sel_key[q2] - mx[q2]) / z[q2];
+              else if (p.gating == 1) wv[q2] = expf(sel_key[q2] - key0[q2]);
+              else wv[q2] = 1.0f / (1.0f + expf(-(p.bias_select_only ? sel_val[q2] : sel_key[q2])));
+            }
+            den[q2] = wv[q2];
+          }
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+            for (int q2 = 0; q2 < R; ++q2) den[q2] += __shfl_xor_sync(0xffffffffu, den[q2], off);
+#pragma unroll
+          for (int q2 = 0; q2 < R; ++q2) {
+            const int64_t grow_r = row0 + rb + q2;
+            if (lane < k && grow_r < p.rows) {
+              p.ids[grow_r * k + lane] = sel_idx[q2];
+              p.wts[grow_r * k + lane] = p.gating == 3 ? wv[q2] : wv[q2] / den[q2];  // rule 3: not renormalised
+            }
           }
         }
-        bool xok = true;
-        if (part == 1) {
-          xok = mbar_wait_bounded(smem_u32(xempty), x_phase ^ 1u, abort_flag, p.wait_limit_ns, p.status);
-          if (xok) {
-#pragma unroll
-            for (int s = 0; s < KMAX; ++s) {
-              x_key[s * 128 + r] = tk.key[s];
-              x_idx[s * 128 + r] = tk.idx[s];
-              x_val[s * 128 + r] = tk.val[s];
-            }
-            x_mx[r] = mx;
-            x_z[r] = z;
-            mbar_arrive(smem_u32(xfull));
-          }
-        } else {
-          xok = mbar_wait_bounded(smem_u32(xfull), x_phase, abort_flag, p.wait_limit_ns, p.status);
-          if (xok) {
-#pragma unroll
-            for (int s = 0; s < KMAX; ++s) tk.push(x_key[s * 128 + r], x_idx[s * 128 + r], x_val[s * 128 + r]);
-            const float mx1 = x_mx[r], z1 = x_z[r];
-            mbar_arrive(smem_u32(xempty));
-            if (all_e) {  // the two partial denominators, brought to the common maximum
-              const float m = fmaxf(mx, mx1);
-              z = z * expf(mx - m) + (z1 > 0.f ? z1 * expf(mx1 - m) : 0.f);
-              mx = m;
-            }
-            if (ok) {
-              float wsel[KMAX];
-              float den = 0.f;
-#pragma unroll
-              for (int s = 0; s < KMAX; ++s) {
-                float wv = 0.f;
-                if (s < p.k) {
-                  if (all_e) wv = expf(tk.key[s] - mx) / z;
-                  else if (p.gating == 1) wv = expf(tk.key[s] - tk.key[0]);
-                  else wv = 1.0f / (1.0f + expf(-(p.bias_select_only ? tk.val[s] : tk.key[s])));
-                }
-                wsel[s] = wv;
-                den += wv;
-              }
-#pragma unroll
-              for (int s = 0; s < KMAX; ++s) {
-                if (s < p.k) {
-                  p.ids[grow * p.k + s] = tk.idx[s];
-                  p.wts[grow * p.k + s] = p.gating == 3 ? wsel[s] : wsel[s] / den;  // rule 3: not renormalised
-                }
-              }
-            }
-          }
-        }
-        x_phase ^= 1u;
-        if (!xok) break;
       }
       tc_fence_before();
       mbar_arrive(smem_u32(&tempty[acc]));
@@ -524,6 +565,9 @@ cudaError_t launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const Para
   if (e != cudaSuccess) return e;
   int64_t grid = device_sm_count();
   if (tiles_bound < grid) grid = tiles_bound;
+  // the router's epilogue stages a tile's logits over the operand ring, so
+  // each CTA takes exactly one tile (tiles_bound is then the tile count)
+  if (MODE == MODE_ROUTER) grid = tiles_bound;
   if (grid < 1) grid = 1;
   grouped_gemm_tc_kernel<MODE, KMAX, FP8><<<(unsigned)grid, kThreads<FP8, MODE>, smem, stream>>>(ta, tb, p);
   return cudaGetLastError();

@@ -25,6 +25,8 @@ struct RouterArgs {
   float* aux_part;
 };
 constexpr int kAuxMaxBlocks = 2048;  // router blocks of a penalty pass, at most
+// Does the router run on the tensor cores (launch_router_topk_tc)?
+inline bool router_uses_tc(bool bf16, int E, int64_t T) { return bf16 && E >= 64 && E <= 256 && T > 64; }
 cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t stream);       // picks one of:
 cudaError_t launch_router_topk_simt(const RouterArgs& a, cudaStream_t stream);  // CUDA cores, any dtype
 cudaError_t launch_router_topk_tc(const RouterArgs& a, cudaStream_t stream);    // tcgen05, bf16, E <= 256
@@ -94,10 +96,10 @@ int64_t decode_counter_cap(int64_t rows, int G, int d, int f);
 // q = e4m3(x / s); rows past *rows_dev (when given) are left alone
 cudaError_t launch_quantize_e4m3(const void* src, int64_t rows, const int32_t* rows_dev, int cols, uint8_t* q,
                                  float* scale, cudaStream_t stream);
-// the same for dispatched rows: output row r quantises x row perm[r] / k
-cudaError_t launch_gather_quantize_e4m3(const void* x, const int32_t* perm, int k, int64_t rows,
-                                        const int32_t* rows_dev, int cols, uint8_t* q, float* scale,
-                                        cudaStream_t stream);
+// the dispatch with 8-bit experts: token t of x [T, cols] quantised once, its
+// codes and scale written to every kept row row_of[t*k + s]
+cudaError_t launch_gather_quantize_e4m3(const void* x, const int32_t* row_of, int k, int64_t T, int cols,
+                                        uint8_t* q, float* scale, cudaStream_t stream);
 inline size_t e4m3_codes_bytes(int64_t rows, int64_t cols) { return ((size_t)(rows * cols) + 255) / 256 * 256; }
 
 // ---- combine (combine.cu)

@@ -26,7 +26,7 @@ int device_sm_count() {
 // the CUDA cores is cheaper than a 128-token tensor tile; a decode-sized batch
 // (at most 64 tokens) gets a block per token on the CUDA cores either way.
 cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t stream) {
-  if (a.bf16 && a.E >= 64 && a.E <= 256 && a.T > 64) return launch_router_topk_tc(a, stream);
+  if (router_uses_tc(a.bf16, a.E, a.T)) return launch_router_topk_tc(a, stream);
   return launch_router_topk_simt(a, stream);
 }
 
@@ -370,16 +370,15 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
   RouterArgs ra{x, w_router, logit_bias, ids, w, cfg->T, cfg->d_model, cfg->n_experts, cfg->top_k,
                 cfg->gating, cfg->bias_select_only, cfg->dtype == MOE_BF16, k.status, wait_limit(cfg)};
   MOE_CUDA_TRY(launch_router_topk(ra, stream));
-  // 8-bit experts: the dispatch writes no bf16 copy; the expert input rows are
-  // quantised straight from x, gathered by perm
+  // 8-bit experts: the dispatch writes no bf16 copy; each token is quantised
+  // once, straight from x, and its codes go to its rows
   const bool e4m3 = cfg->weight_format == MOE_W_E4M3;
   PermuteArgs pa{ids, x, counts, k.offsets, k.perm, k.row_of, e4m3 ? nullptr : k.x_perm, k.chunk_counts,
                  cfg->T * cfg->top_k, cfg->top_k, cfg->d_model, cfg->n_experts, (int)elem_bytes(cfg), k.status,
                  capacity_rows(cfg)};
   MOE_CUDA_TRY(launch_permute(pa, stream));
   if (e4m3)
-    MOE_CUDA_TRY(launch_gather_quantize_e4m3(x, k.perm, cfg->top_k, cfg->T * cfg->top_k, k.offsets + cfg->n_experts,
-                                             cfg->d_model, k.xq, k.sx, stream));
+    MOE_CUDA_TRY(launch_gather_quantize_e4m3(x, k.row_of, cfg->top_k, cfg->T, cfg->d_model, k.xq, k.sx, stream));
   MOE_CUDA_TRY(run_ffn(cfg, k, k.x_perm, k.offsets, cfg->n_experts, cfg->T * cfg->top_k, cfg->d_ff, w_gate_up,
                        w_down, k.h, k.y_perm, stream, false, e4m3));
   if (cfg->n_shared > 0)

@@ -227,27 +227,34 @@ __global__ void __launch_bounds__(kSmallThreads)
   }
 }
 
-// x_perm[row] = x[perm[row] / k]; one warp per row, 16-byte vectors
+// x_perm[row_of[t*k + s]] = x[t] for every kept slot s of token t.  Token
+// major: one warp per token reads the token's vector once (16-byte vectors,
+// four in flight per lane) and writes it to each of its rows, so x crosses
+// HBM once however many experts a token picked (walking the rows in dispatch
+// order instead re-reads x from HBM once its k copies have pushed it out of L2).
 __global__ void __launch_bounds__(kThreads) gather_rows_kernel(const uint8_t* __restrict__ x,
-                                                               const int32_t* __restrict__ perm,
-                                                               const int32_t* __restrict__ offsets, int E,
+                                                               const int32_t* __restrict__ row_of, int64_t T,
                                                                int k, int64_t row_bytes, uint8_t* x_perm) {
-  const int64_t n_rows = offsets[E];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t n16 = row_bytes / 16;
-  for (int64_t row = (int64_t)blockIdx.x * kWarps + warp; row < n_rows; row += (int64_t)gridDim.x * kWarps) {
-    const int64_t t = perm[row] / k;
+  for (int64_t t = (int64_t)blockIdx.x * kWarps + warp; t < T; t += (int64_t)gridDim.x * kWarps) {
+    const int my_row = lane < k ? row_of[t * k + lane] : -1;  // k <= kMaxTopK <= 32
     const uint4* src = reinterpret_cast<const uint4*>(x + t * row_bytes);
-    uint4* dst = reinterpret_cast<uint4*>(x_perm + row * row_bytes);
-    int64_t j = lane;
-    for (; j + 96 < n16; j += 128) {  // four independent 16-byte loads in flight per lane
-      const uint4 a0 = __ldg(src + j), a1 = __ldg(src + j + 32), a2 = __ldg(src + j + 64), a3 = __ldg(src + j + 96);
-      dst[j] = a0;
-      dst[j + 32] = a1;
-      dst[j + 64] = a2;
-      dst[j + 96] = a3;
+    for (int64_t j0 = 0; j0 < n16; j0 += 128) {  // the same trip count on every lane (shuffles inside)
+      const int64_t j = j0 + lane;
+      uint4 a[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (j + 32 * i < n16) a[i] = __ldg(src + j + 32 * i);
+      for (int s = 0; s < k; ++s) {
+        const int row = __shfl_sync(0xffffffffu, my_row, s);
+        if (row < 0) continue;  // dropped by the capacity
+        uint4* dst = reinterpret_cast<uint4*>(x_perm + (int64_t)row * row_bytes);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (j + 32 * i < n16) dst[j + 32 * i] = a[i];
+      }
     }
-    for (; j < n16; j += 32) dst[j] = __ldg(src + j);
   }
 }
 
@@ -276,11 +283,12 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || a.x == nullptr || a.x_perm == nullptr) return e;
-  int64_t blocks = (a.n_assign + kWarps - 1) / kWarps;
+  const int64_t T = a.n_assign / a.k;
+  int64_t blocks = (T + kWarps - 1) / kWarps;
   const int64_t cap = (int64_t)device_sm_count() * 16;
   if (blocks > cap) blocks = cap;
   gather_rows_kernel<<<(unsigned)blocks, kThreads, 0, stream>>>(
-      static_cast<const uint8_t*>(a.x), a.perm, a.offsets, a.E, a.k, (int64_t)a.d * a.elem_bytes,
+      static_cast<const uint8_t*>(a.x), a.row_of, T, a.k, (int64_t)a.d * a.elem_bytes,
       static_cast<uint8_t*>(a.x_perm));
   return cudaGetLastError();
 }

@@ -12,10 +12,9 @@
 // IEEE-rounded fp32 division and the hardware fp32 -> e4m3 conversion.
 //
 // One warp per row; eight values per lane leave as one 8-byte word.  The
-// dispatch path quantises while it gathers: output row r is the token row
-// perm[r] / k, so each dispatched copy is quantised straight from x (the same
-// codes as quantising the gathered bf16 copy) and the bf16 copy is never
-// written.
+// dispatch path quantises while it gathers: each token's vector is quantised
+// once, straight from x, and its codes are written to the token's rows (the
+// same codes as quantising the gathered bf16 copies, which are never written).
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -59,26 +58,21 @@ __device__ __forceinline__ float row_scale(float amax) {
   return amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
 }
 
-// Output row r reads source row perm[r] / k (a dispatched copy of a token's
-// vector) when perm is given, else row r.  Rows past *rows_dev (when given)
-// are left alone.
-
-// A pass for the absolute maximum, then a pass that converts (it finds the
-// row in L1).  Four independent 16-byte loads in flight per lane; 40
-// registers, so that many warps per SM hide the latency of the loads and of
-// the IEEE divisions (a variant holding the whole row in registers ran at
-// one block per SM and measured slower).
+// Row r of src -> codes row r and scale[r]; rows past *rows_dev (when given)
+// are left alone.  A pass for the absolute maximum, then a pass that converts
+// (it finds the row in L1).  Four independent 16-byte loads in flight per
+// lane; 40 registers, so that many warps per SM hide the latency of the loads
+// and of the IEEE divisions (a variant holding the whole row in registers ran
+// at one block per SM and measured slower).
 __global__ void __launch_bounds__(kThreads)
-    quantize_rows_e4m3_kernel(const __nv_bfloat16* __restrict__ src, const int32_t* __restrict__ perm, int k,
-                              int64_t rows, const int32_t* rows_dev, int cols, uint8_t* __restrict__ q,
-                              float* __restrict__ scale) {
+    quantize_rows_e4m3_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, const int32_t* rows_dev,
+                              int cols, uint8_t* __restrict__ q, float* __restrict__ scale) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t dr = rows_dev ? (int64_t)*rows_dev : rows;
   const int64_t n = dr < rows ? dr : rows;
   const int nv = cols / 8;
   for (int64_t r = (int64_t)blockIdx.x * kWarps + warp; r < n; r += (int64_t)gridDim.x * kWarps) {
-    const int64_t sr = perm ? (int64_t)(perm[r] / k) : r;
-    const uint4* row = reinterpret_cast<const uint4*>(src + sr * cols);
+    const uint4* row = reinterpret_cast<const uint4*>(src + r * cols);
     float amax = 0.f;
     int v = lane;
     for (; v + 96 < nv; v += 128) {  // four independent loads in flight per lane
@@ -100,28 +94,66 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-cudaError_t launch_rows(const void* src, const int32_t* perm, int k, int64_t rows, const int32_t* rows_dev, int cols,
-                        uint8_t* q, float* scale, cudaStream_t stream) {
-  if (rows == 0) return cudaSuccess;
-  int64_t blocks = (rows + kWarps - 1) / kWarps;
+// The dispatch with 8-bit experts: token t of x is quantised once and its
+// codes and scale go to every kept row row_of[t*k + s] (one warp per token,
+// as in the bf16 gather), so x crosses HBM once and no bf16 copy is written.
+__global__ void __launch_bounds__(kThreads)
+    gather_quantize_e4m3_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ row_of,
+                                int64_t T, int k, int cols, uint8_t* __restrict__ q, float* __restrict__ scale) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int nv = cols / 8;
+  for (int64_t t = (int64_t)blockIdx.x * kWarps + warp; t < T; t += (int64_t)gridDim.x * kWarps) {
+    const uint4* row = reinterpret_cast<const uint4*>(x + t * cols);
+    const int my_row = lane < k ? row_of[t * k + lane] : -1;  // k <= kMaxTopK <= 32
+    float amax = 0.f;
+    int v = lane;
+    for (; v + 96 < nv; v += 128) {
+      const uint4 a0 = __ldg(row + v), a1 = __ldg(row + v + 32), a2 = __ldg(row + v + 64), a3 = __ldg(row + v + 96);
+      amax = amax8(a3, amax8(a2, amax8(a1, amax8(a0, amax))));
+    }
+    for (; v < nv; v += 32) amax = amax8(__ldg(row + v), amax);
+    const float s = row_scale(amax);
+    if (my_row >= 0) scale[my_row] = s;
+    for (int v0 = 0; v0 < nv; v0 += 128) {  // the same trip count on every lane (shuffles inside)
+      v = v0 + lane;
+      uint2 c[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (v + 32 * i < nv) c[i] = e4m3x8(__ldg(row + v + 32 * i), s);
+      for (int j = 0; j < k; ++j) {
+        const int r = __shfl_sync(0xffffffffu, my_row, j);
+        if (r < 0) continue;  // dropped by the capacity
+        uint2* out = reinterpret_cast<uint2*>(q + (int64_t)r * cols);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (v + 32 * i < nv) out[v + 32 * i] = c[i];
+      }
+    }
+  }
+}
+
+int64_t grid_for(int64_t units) {
+  int64_t blocks = (units + kWarps - 1) / kWarps;
   const int64_t cap = (int64_t)device_sm_count() * 16;
-  if (blocks > cap) blocks = cap;
-  const auto* x = static_cast<const __nv_bfloat16*>(src);
-  quantize_rows_e4m3_kernel<<<(unsigned)blocks, kThreads, 0, stream>>>(x, perm, k, rows, rows_dev, cols, q, scale);
-  return cudaGetLastError();
+  return blocks > cap ? cap : blocks;
 }
 
 }  // namespace
 
 cudaError_t launch_quantize_e4m3(const void* src, int64_t rows, const int32_t* rows_dev, int cols, uint8_t* q,
                                  float* scale, cudaStream_t stream) {
-  return launch_rows(src, nullptr, 1, rows, rows_dev, cols, q, scale, stream);
+  if (rows == 0) return cudaSuccess;
+  quantize_rows_e4m3_kernel<<<(unsigned)grid_for(rows), kThreads, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(src), rows, rows_dev, cols, q, scale);
+  return cudaGetLastError();
 }
 
-cudaError_t launch_gather_quantize_e4m3(const void* x, const int32_t* perm, int k, int64_t rows,
-                                        const int32_t* rows_dev, int cols, uint8_t* q, float* scale,
-                                        cudaStream_t stream) {
-  return launch_rows(x, perm, k, rows, rows_dev, cols, q, scale, stream);
+cudaError_t launch_gather_quantize_e4m3(const void* x, const int32_t* row_of, int k, int64_t T, int cols,
+                                        uint8_t* q, float* scale, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  gather_quantize_e4m3_kernel<<<(unsigned)grid_for(T), kThreads, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(x), row_of, T, k, cols, q, scale);
+  return cudaGetLastError();
 }
 
 }  // namespace moe

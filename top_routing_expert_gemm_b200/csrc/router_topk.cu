@@ -168,7 +168,7 @@ template <typename T, bool W_SMEM, int KMAX, bool AUX>
 __global__ void __launch_bounds__(kThreads) router_topk_simt_kernel(RouterParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int V = Vec16<T>::N;
-  const int d = p.d, E = p.E, k = p.k;
+  const int d = p.d, E = p.E;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const T* __restrict__ x = static_cast<const T*>(p.x);
   const T* __restrict__ wg = static_cast<const T*>(p.w);
