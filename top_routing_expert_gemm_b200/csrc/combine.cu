@@ -3,7 +3,8 @@
 // and VRAM" (step 5: multiply each expert output by its weight and add them
 // up); "Mixture of Experts: why a model with 671 billion parameters uses only
 // 37" ("Where MoE changes the Transformer": outputs summed, weighted by the
-// router's scores).  One block per token, 16-byte vectors, fp32 accumulation.
+// router's scores).  One block per token, 16-byte vectors, fp32 accumulation
+// in slot order.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -12,7 +13,10 @@ namespace {
 
 constexpr int kThreads = 128;
 
-template <typename T>
+// KMAX >= k: the k rows of a token are read with independent loads (the slot
+// loop is unrolled), so each thread has k 16-byte loads in flight instead of
+// one; the token's rows and weights are read once per thread.
+template <typename T, int KMAX>
 __global__ void __launch_bounds__(kThreads) combine_kernel(const T* __restrict__ y_perm,
                                                            const int32_t* __restrict__ row_of,
                                                            const float* __restrict__ w,
@@ -21,17 +25,27 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const T* __restrict__
   constexpr int V = Vec16<T>::N;
   const int nv = d / V;
   for (int64_t t = blockIdx.x; t < n_tok; t += gridDim.x) {
+    int rows[KMAX];
+    float ws[KMAX];
+#pragma unroll
+    for (int s = 0; s < KMAX; ++s) {
+      rows[s] = s < k ? row_of[t * k + s] : -1;
+      ws[s] = s < k ? w[t * k + s] : 0.f;
+    }
     for (int v = threadIdx.x; v < nv; v += kThreads) {
+      Vec16<T> yv[KMAX];
+#pragma unroll
+      for (int s = 0; s < KMAX; ++s)
+        if (rows[s] >= 0) yv[s] = ld16(y_perm + (int64_t)rows[s] * d + (int64_t)v * V);
       float acc[V];
 #pragma unroll
       for (int j = 0; j < V; ++j) acc[j] = 0.f;
-      for (int s = 0; s < k; ++s) {
-        const int row = row_of[t * k + s];
-        if (row < 0) continue;
-        const float ws = w[t * k + s];
-        const Vec16<T> yv = ld16(y_perm + (int64_t)row * d + (int64_t)v * V);
 #pragma unroll
-        for (int j = 0; j < V; ++j) acc[j] = fmaf(ws, Elem<T>::to_f(yv.v[j]), acc[j]);
+      for (int s = 0; s < KMAX; ++s) {  // slot order: the same sums as a plain loop over s
+        if (rows[s] >= 0) {
+#pragma unroll
+          for (int j = 0; j < V; ++j) acc[j] = fmaf(ws[s], Elem<T>::to_f(yv[s].v[j]), acc[j]);
+        }
       }
       if (y_shared) {
         const Vec16<T> sv = ld16(y_shared + t * d + (int64_t)v * V);
@@ -46,6 +60,18 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const T* __restrict__
   }
 }
 
+template <typename T>
+cudaError_t launch_t(const CombineArgs& a, unsigned blocks, cudaStream_t stream) {
+  const T* yp = static_cast<const T*>(a.y_perm);
+  const T* ys = static_cast<const T*>(a.y_shared);
+  T* y = static_cast<T*>(a.y);
+  if (a.k <= 2) combine_kernel<T, 2><<<blocks, kThreads, 0, stream>>>(yp, a.row_of, a.w, ys, y, a.T, a.k, a.d);
+  else if (a.k <= 4) combine_kernel<T, 4><<<blocks, kThreads, 0, stream>>>(yp, a.row_of, a.w, ys, y, a.T, a.k, a.d);
+  else if (a.k <= 8) combine_kernel<T, 8><<<blocks, kThreads, 0, stream>>>(yp, a.row_of, a.w, ys, y, a.T, a.k, a.d);
+  else combine_kernel<T, kMaxTopK><<<blocks, kThreads, 0, stream>>>(yp, a.row_of, a.w, ys, y, a.T, a.k, a.d);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream) {
@@ -53,16 +79,7 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream) {
   int64_t blocks = a.T;
   const int64_t cap = (int64_t)device_sm_count() * 64;
   if (blocks > cap) blocks = cap;
-  if (a.bf16) {
-    combine_kernel<__nv_bfloat16><<<(unsigned)blocks, kThreads, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(a.y_perm), a.row_of, a.w,
-        static_cast<const __nv_bfloat16*>(a.y_shared), static_cast<__nv_bfloat16*>(a.y), a.T, a.k, a.d);
-  } else {
-    combine_kernel<float><<<(unsigned)blocks, kThreads, 0, stream>>>(
-        static_cast<const float*>(a.y_perm), a.row_of, a.w, static_cast<const float*>(a.y_shared),
-        static_cast<float*>(a.y), a.T, a.k, a.d);
-  }
-  return cudaGetLastError();
+  return a.bf16 ? launch_t<__nv_bfloat16>(a, (unsigned)blocks, stream) : launch_t<float>(a, (unsigned)blocks, stream);
 }
 
 }  // namespace moe
