@@ -38,28 +38,33 @@ METRIC = "MoE-layer tokens/s (active TFLOP/s and roofline fraction alongside)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-GEMM_SOURCES = ("grouped_gemm_tc.cu", "grouped_gemm_swap.cu", "tc_primitives.cuh", "common.cuh", "kernels.cuh")
+# the sources of the expert GEMMs of each schedule (token-rows-as-M kernel for
+# large batches, swapped-operand kernel for the decode regime)
+GEMM_SOURCES = {
+    "tc": ("grouped_gemm_tc.cu", "tc_primitives.cuh", "common.cuh", "kernels.cuh"),
+    "decode": ("grouped_gemm_swap.cu", "tc_primitives.cuh", "common.cuh", "kernels.cuh"),
+}
 TRAFFIC_FILE = ROOT / "profiles" / "dram_traffic.json"
 
 
-def gemm_sources_sha256() -> str:
-    """Digest of the expert-GEMM kernel sources: a DRAM-traffic record taken
-    with ncu applies only while this matches."""
+def gemm_sources_sha256(schedule: str) -> str:
+    """Digest of the expert-GEMM kernel sources of a schedule: a DRAM-traffic
+    record taken with ncu applies only while this matches."""
     import hashlib
 
     h = hashlib.sha256()
-    for name in GEMM_SOURCES:
+    for name in GEMM_SOURCES[schedule]:
         h.update((ROOT / "top_routing_expert_gemm_b200" / "csrc" / name).read_bytes())
     return h.hexdigest()
 
 
-def recorded_traffic(workload: str):
+def recorded_traffic(workload: str, schedule: str):
     """DRAM bytes (read + write) per step of the expert GEMMs from the committed
     ncu record, or None when there is none or the kernels changed since."""
     if not TRAFFIC_FILE.exists():
         return None
     rec = json.loads(TRAFFIC_FILE.read_text()).get(workload)
-    if not rec or rec.get("gemm_sources_sha256") != gemm_sources_sha256():
+    if not rec or rec.get("gemm_sources_sha256") != gemm_sources_sha256(schedule):
         return None
     return rec.get("bytes_per_step")
 
@@ -540,7 +545,7 @@ def main() -> None:
         kname = "grouped_gemm_tc_kernel (token rows as M)"
     roof["kernel"] = (kname + ": the GEMM-1 and GEMM-2 launches of moe_grouped_ffn"
                       + (" (routed and shared experts)" if cfg.n_shared else ""))
-    roof["traffic"] = recorded_traffic(cfg.name)
+    roof["traffic"] = recorded_traffic(cfg.name, "decode" if uses_decode_schedule(cfg) else "tc")
     roof["peak_source"] = pk_kind + (" bf16 x 2 (nominal fp8/bf16 dense ratio)" if cfg.e4m3 and not decode else "")
     line = {
         "metric": METRIC,
