@@ -42,7 +42,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # large batches, swapped-operand kernel for the decode regime)
 GEMM_SOURCES = {
     "tc": ("grouped_gemm_tc.cu", "tc_primitives.cuh", "common.cuh", "kernels.cuh"),
-    "decode": ("grouped_gemm_swap.cu", "tc_primitives.cuh", "common.cuh", "kernels.cuh"),
+    "decode": ("grouped_gemm_swap.cu", "tc_primitives.cuh", "pdl.cuh", "common.cuh", "kernels.cuh"),
 }
 TRAFFIC_FILE = ROOT / "profiles" / "dram_traffic.json"
 

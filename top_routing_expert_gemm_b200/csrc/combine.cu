@@ -7,6 +7,7 @@
 // in slot order.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "pdl.cuh"
 
 namespace moe {
 namespace {
@@ -24,6 +25,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const T* __restrict__
                                                            int64_t n_tok, int k, int d) {
   constexpr int V = Vec16<T>::N;
   const int nv = d / V;
+  grid_dependency_wait();  // the expert outputs (programmatic launch)
   for (int64_t t = blockIdx.x; t < n_tok; t += gridDim.x) {
     int rows[KMAX];
     float ws[KMAX];
@@ -65,11 +67,14 @@ cudaError_t launch_t(const CombineArgs& a, unsigned blocks, cudaStream_t stream)
   const T* yp = static_cast<const T*>(a.y_perm);
   const T* ys = static_cast<const T*>(a.y_shared);
   T* y = static_cast<T*>(a.y);
-  if (a.k <= 2) combine_kernel<T, 2><<<blocks, kThreads, 0, stream>>>(yp, a.row_of, a.w, ys, y, a.T, a.k, a.d);
-  else if (a.k <= 4) combine_kernel<T, 4><<<blocks, kThreads, 0, stream>>>(yp, a.row_of, a.w, ys, y, a.T, a.k, a.d);
-  else if (a.k <= 8) combine_kernel<T, 8><<<blocks, kThreads, 0, stream>>>(yp, a.row_of, a.w, ys, y, a.T, a.k, a.d);
-  else combine_kernel<T, kMaxTopK><<<blocks, kThreads, 0, stream>>>(yp, a.row_of, a.w, ys, y, a.T, a.k, a.d);
-  return cudaGetLastError();
+  auto run = [&](auto kernel) {
+    return launch_maybe_chained(kernel, dim3(blocks), dim3(kThreads), 0, stream, a.chained, yp, a.row_of, a.w, ys, y,
+                                a.T, a.k, a.d);
+  };
+  if (a.k <= 2) return run(combine_kernel<T, 2>);
+  if (a.k <= 4) return run(combine_kernel<T, 4>);
+  if (a.k <= 8) return run(combine_kernel<T, 8>);
+  return run(combine_kernel<T, kMaxTopK>);
 }
 
 }  // namespace

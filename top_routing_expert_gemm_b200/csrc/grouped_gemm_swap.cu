@@ -48,6 +48,7 @@
 #include <cmath>
 
 #include "kernels.cuh"
+#include "pdl.cuh"
 #include "tc_primitives.cuh"
 
 namespace moe {
@@ -93,13 +94,6 @@ struct SwapParams {
 size_t swap_smem_bytes(int G) {
   return 1024 + (size_t)STAGES * (S_A_BYTES + B_BYTES) + S_STAGE_BYTES + 256 + 2 * sizeof(int) * (size_t)(G + 1);
 }
-
-// Programmatic launch: let the next grid of the stream (launched with
-// programmatic serialisation) be scheduled before this one finishes; wait
-// until the grids this one depends on have finished and their memory
-// operations are visible (at once for a launch without the attribute).
-__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // Named barrier of the four epilogue warps (barrier 1, 128 threads).
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
@@ -251,14 +245,13 @@ __global__ void __launch_bounds__(S_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // Programmatic launch: GEMM-1 lets GEMM-2 be scheduled now (its CTAs take
-  // the SMs this grid frees), and GEMM-2 waits here, after its set-up, until
-  // everything before it in the stream has finished and its writes are
-  // visible; both are no-ops for a launch without the attribute.  Everything
-  // above reads only what earlier launches finished before this grid began
-  // (the offsets of the dispatch).
-  if (threadIdx.x == 0) grid_launch_dependents();
+  // Programmatic launch (pdl.cuh): wait here, after the set-up, for the
+  // predecessor (GEMM-1 for GEMM-2, the gather for GEMM-1 of a chained layer
+  // step), then let the successor be scheduled: its CTAs take the SMs this
+  // grid frees.  The set-up above reads only the offsets of the dispatch,
+  // which finished before the predecessor passed its own wait.
   grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
 
   const uint32_t tmem_base = *tmem_slot;
   constexpr int KB = FP8 ? 2 * S_BK : S_BK;  // elements per 128-byte K slice
@@ -511,36 +504,25 @@ __global__ void __launch_bounds__(S_THREADS, 1)
   }
 }
 
-// after_gemm1: the launch follows GEMM-1 (directly, or behind the 8-bit
-// re-quantisation of h) and is programmatic: it may be scheduled while its
-// predecessor drains and waits in the kernel for it to finish; its counters
-// are the ones GEMM-1 left at zero (each unit's last contributor resets its
-// counter), so no clearing launch sits in between.  Otherwise the counters are
-// cleared first (a launch that timed out may leave some set).
+// chained: the launch is programmatic (pdl.cuh) and finds its unit counters at
+// zero: GEMM-2 after GEMM-1 (directly, or behind the 8-bit re-quantisation
+// of h), whose units' last contributors reset every counter they used, or
+// GEMM-1 of a layer step that cleared the counters ahead (moe_forward).
+// Otherwise the counters are cleared first (a launch that timed out may leave
+// some set).
 template <int EPI, bool FP8>
 cudaError_t launch_swap(const CUtensorMap& tw, const CUtensorMap& tx64, const CUtensorMap& tx16,
-                        const SwapParams& p, int grid, bool after_gemm1, cudaStream_t stream) {
+                        const SwapParams& p, int grid, bool chained, cudaStream_t stream) {
   auto kernel = grouped_gemm_swap_kernel<EPI, FP8>;
   const size_t smem = swap_smem_bytes(p.G);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  if (!after_gemm1) {
+  if (!chained) {
     e = cudaMemsetAsync(p.counters, 0, sizeof(int) * (size_t)p.counter_cap, stream);
     if (e != cudaSuccess) return e;
-    kernel<<<(unsigned)grid, S_THREADS, smem, stream>>>(tw, tx64, tx16, p);
-    return cudaGetLastError();
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(S_THREADS);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, tw, tx64, tx16, p);
+  return launch_maybe_chained(kernel, dim3((unsigned)grid), dim3(S_THREADS), smem, stream, chained, tw, tx64, tx16,
+                              p);
 }
 
 // Units of one GEMM, bounded from the row count (the chunking is per group).
@@ -572,8 +554,8 @@ cudaError_t run_swap(const GroupedFfnArgs& a, cudaStream_t stream) {
     return cudaErrorInvalidValue;
   SwapParams p1{a.offsets, G, a.rows, a.d, a.f, J1, w1_rows, a.f, static_cast<__nv_bfloat16*>(a.h), a.f,
                 a.partial, a.counters, a.counter_cap, a.status, lim, a.sa, s1};
-  cudaError_t e = gelu ? launch_swap<kEpiGELU, FP8>(w1, x1a, x1b, p1, grid, false, stream)
-                       : launch_swap<kEpiSwiGLU, FP8>(w1, x1a, x1b, p1, grid, false, stream);
+  cudaError_t e = gelu ? launch_swap<kEpiGELU, FP8>(w1, x1a, x1b, p1, grid, a.chained, stream)
+                       : launch_swap<kEpiSwiGLU, FP8>(w1, x1a, x1b, p1, grid, a.chained, stream);
   if (e != cudaSuccess) return e;
   const void* b2 = a.h;
   const float* sx2 = nullptr;

@@ -49,6 +49,7 @@ struct PermuteArgs {
   int elem_bytes;
   int* status;
   int64_t capacity;       // rows each expert keeps (n_assign or more: dropless)
+  bool chained;           // the dispatch kernels may be launched programmatically (pdl.cuh)
 };
 int permute_n_chunks(int64_t n_assign);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream);
@@ -81,6 +82,9 @@ struct GroupedFfnArgs {
   int64_t partial_slots;
   int* counters;
   int64_t counter_cap;
+  // decode kernel: the counters were zeroed ahead of this call, so GEMM-1 is
+  // launched programmatically after its predecessor (pdl.cuh) with no clearing
+  bool chained;
 };
 constexpr int kDecodeMaxCtas = 160;  // CTAs of one decode-schedule launch, at most
 constexpr int kDecodeTokens = 64;    // most tokens per unit of the decode schedule
@@ -99,7 +103,7 @@ cudaError_t launch_quantize_e4m3(const void* src, int64_t rows, const int32_t* r
 // the dispatch with 8-bit experts: token t of x [T, cols] quantised once, its
 // codes and scale written to every kept row row_of[t*k + s]
 cudaError_t launch_gather_quantize_e4m3(const void* x, const int32_t* row_of, int k, int64_t T, int cols,
-                                        uint8_t* q, float* scale, cudaStream_t stream);
+                                        uint8_t* q, float* scale, bool chained, cudaStream_t stream);
 inline size_t e4m3_codes_bytes(int64_t rows, int64_t cols) { return ((size_t)(rows * cols) + 255) / 256 * 256; }
 
 // ---- combine (combine.cu)
@@ -112,6 +116,7 @@ struct CombineArgs {
   int64_t T;
   int k, d;
   bool bf16;
+  bool chained;  // may be launched programmatically after the expert GEMMs (pdl.cuh)
 };
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
 

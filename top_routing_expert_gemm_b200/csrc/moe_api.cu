@@ -181,12 +181,15 @@ moe_status bind(const void* p) {
 
 uint64_t wait_limit(const moe_config* c) { return c->wait_limit_ns > 0 ? (uint64_t)c->wait_limit_ns : 2000000000ull; }
 
-// a_quantized: 8-bit experts whose input rows are already in xq / sx
+// a_quantized: 8-bit experts whose input rows are already in xq / sx;
+// chained: a layer step that cleared the decode counters ahead and chains its
+// launches (pdl.cuh)
 cudaError_t run_ffn(const moe_config* c, const Carve& k, const void* a, const int32_t* offsets, int G, int64_t rows,
                     int f, const void* w_gu, const void* w_d, void* h, void* y, cudaStream_t s, bool shared = false,
-                    bool a_quantized = false) {
+                    bool a_quantized = false, bool chained = false) {
   GroupedFfnArgs g{a, offsets, w_gu, w_d, h, y, rows, G, c->d_model, f, c->expert_act, k.status, wait_limit(c),
-                   false, nullptr, nullptr, nullptr, k.partial, k.partial_slots, k.counters, k.counter_cap};
+                   false, nullptr, nullptr, nullptr, k.partial, k.partial_slots, k.counters, k.counter_cap,
+                   chained};
   if (c->dtype != MOE_BF16) return launch_grouped_ffn_f32_simt(g, s);
   if (c->weight_format == MOE_W_E4M3) {
     // the expert input -> E4M3 codes and per-token scales (only the rows in use)
@@ -364,6 +367,11 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
   if ((st = bind(x)) != MOE_OK) return st;
   Carve k = carve(cfg, ws);
   MOE_CUDA_TRY(cudaMemsetAsync(k.status, 0, 16, stream));
+  // The launches of the step are chained (pdl.cuh): each kernel after the
+  // router may be scheduled while its predecessor finishes.  The decode
+  // kernels' unit counters are cleared here, ahead of the chain, instead of
+  // by a clearing launch in front of GEMM-1.
+  if (k.counters) MOE_CUDA_TRY(cudaMemsetAsync(k.counters, 0, sizeof(int) * (size_t)k.counter_cap, stream));
   int32_t* ids = opt_topk_ids ? opt_topk_ids : k.ids;
   float* w = opt_topk_w ? opt_topk_w : k.w;
   int32_t* counts = opt_counts ? opt_counts : k.counts;
@@ -375,17 +383,18 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
   const bool e4m3 = cfg->weight_format == MOE_W_E4M3;
   PermuteArgs pa{ids, x, counts, k.offsets, k.perm, k.row_of, e4m3 ? nullptr : k.x_perm, k.chunk_counts,
                  cfg->T * cfg->top_k, cfg->top_k, cfg->d_model, cfg->n_experts, (int)elem_bytes(cfg), k.status,
-                 capacity_rows(cfg)};
+                 capacity_rows(cfg), true};
   MOE_CUDA_TRY(launch_permute(pa, stream));
   if (e4m3)
-    MOE_CUDA_TRY(launch_gather_quantize_e4m3(x, k.row_of, cfg->top_k, cfg->T, cfg->d_model, k.xq, k.sx, stream));
-  MOE_CUDA_TRY(run_ffn(cfg, k, k.x_perm, k.offsets, cfg->n_experts, cfg->T * cfg->top_k, cfg->d_ff, w_gate_up,
-                       w_down, k.h, k.y_perm, stream, false, e4m3));
-  if (cfg->n_shared > 0)
     MOE_CUDA_TRY(
-        run_ffn(cfg, k, x, nullptr, 1, cfg->T, cfg->d_ff_shared, ws_gate_up, ws_down, k.h_s, k.y_s, stream, true));
+        launch_gather_quantize_e4m3(x, k.row_of, cfg->top_k, cfg->T, cfg->d_model, k.xq, k.sx, true, stream));
+  MOE_CUDA_TRY(run_ffn(cfg, k, k.x_perm, k.offsets, cfg->n_experts, cfg->T * cfg->top_k, cfg->d_ff, w_gate_up,
+                       w_down, k.h, k.y_perm, stream, false, e4m3, true));
+  if (cfg->n_shared > 0)
+    MOE_CUDA_TRY(run_ffn(cfg, k, x, nullptr, 1, cfg->T, cfg->d_ff_shared, ws_gate_up, ws_down, k.h_s, k.y_s, stream,
+                         true, false, true));
   CombineArgs ca{k.y_perm, k.row_of, w, cfg->n_shared > 0 ? k.y_s : nullptr, y, cfg->T, cfg->top_k,
-                 cfg->d_model, cfg->dtype == MOE_BF16};
+                 cfg->d_model, cfg->dtype == MOE_BF16, true};
   MOE_CUDA_TRY(launch_combine(ca, stream));
   return MOE_OK;
 }

@@ -23,6 +23,7 @@
 // and a gather kernel that moves whole rows with 16-byte loads/stores.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "pdl.cuh"
 
 namespace moe {
 namespace {
@@ -163,6 +164,8 @@ __global__ void __launch_bounds__(kSmallThreads)
   int* base = sm + E;
   int* run = sm + 2 * E;
   const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+  grid_dependency_wait();  // the router's ids (programmatic launch)
+  if (tid == 0) grid_launch_dependents();
   for (int e = tid; e < E; e += kSmallThreads) {
     hist[e] = 0;
     run[e] = 0;
@@ -237,6 +240,8 @@ __global__ void __launch_bounds__(kThreads) gather_rows_kernel(const uint8_t* __
                                                                int k, int64_t row_bytes, uint8_t* x_perm) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t n16 = row_bytes / 16;
+  grid_dependency_wait();  // row_of of the dispatch (programmatic launch)
+  if (threadIdx.x == 0) grid_launch_dependents();
   for (int64_t t = (int64_t)blockIdx.x * kWarps + warp; t < T; t += (int64_t)gridDim.x * kWarps) {
     const int my_row = lane < k ? row_of[t * k + lane] : -1;  // k <= kMaxTopK <= 32
     const uint4* src = reinterpret_cast<const uint4*>(x + t * row_bytes);
@@ -271,8 +276,10 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
     return cudaMemsetAsync(a.offsets, 0, sizeof(int32_t) * (a.E + 1), stream);
   }
   if (a.n_assign <= kSmallDispatch) {
-    permute_small_kernel<<<1, kSmallThreads, 3 * sizeof(int) * a.E, stream>>>(
-        a.ids, a.n_assign, a.E, a.capacity, a.counts, a.offsets, a.perm, a.row_of, a.status);
+    const cudaError_t e = launch_maybe_chained(permute_small_kernel, dim3(1), dim3(kSmallThreads),
+                                               3 * sizeof(int) * a.E, stream, a.chained, a.ids, a.n_assign, a.E,
+                                               a.capacity, a.counts, a.offsets, a.perm, a.row_of, a.status);
+    if (e != cudaSuccess) return e;
   } else {
     permute_count_kernel<<<n_chunks, kThreads, sizeof(int) * a.E, stream>>>(a.ids, a.n_assign, a.E,
                                                                             a.chunk_counts, n_chunks, a.status);
@@ -287,10 +294,9 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
   int64_t blocks = (T + kWarps - 1) / kWarps;
   const int64_t cap = (int64_t)device_sm_count() * 16;
   if (blocks > cap) blocks = cap;
-  gather_rows_kernel<<<(unsigned)blocks, kThreads, 0, stream>>>(
-      static_cast<const uint8_t*>(a.x), a.row_of, T, a.k, (int64_t)a.d * a.elem_bytes,
-      static_cast<uint8_t*>(a.x_perm));
-  return cudaGetLastError();
+  return launch_maybe_chained(gather_rows_kernel, dim3((unsigned)blocks), dim3(kThreads), 0, stream, a.chained,
+                              static_cast<const uint8_t*>(a.x), a.row_of, T, a.k, (int64_t)a.d * a.elem_bytes,
+                              static_cast<uint8_t*>(a.x_perm));
 }
 
 }  // namespace moe

@@ -19,6 +19,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "pdl.cuh"
 
 namespace moe {
 namespace {
@@ -102,6 +103,8 @@ __global__ void __launch_bounds__(kThreads)
                                 int64_t T, int k, int cols, uint8_t* __restrict__ q, float* __restrict__ scale) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int nv = cols / 8;
+  grid_dependency_wait();  // row_of of the dispatch (programmatic launch)
+  if (threadIdx.x == 0) grid_launch_dependents();
   for (int64_t t = (int64_t)blockIdx.x * kWarps + warp; t < T; t += (int64_t)gridDim.x * kWarps) {
     const uint4* row = reinterpret_cast<const uint4*>(x + t * cols);
     const int my_row = lane < k ? row_of[t * k + lane] : -1;  // k <= kMaxTopK <= 32
@@ -149,11 +152,10 @@ cudaError_t launch_quantize_e4m3(const void* src, int64_t rows, const int32_t* r
 }
 
 cudaError_t launch_gather_quantize_e4m3(const void* x, const int32_t* row_of, int k, int64_t T, int cols,
-                                        uint8_t* q, float* scale, cudaStream_t stream) {
+                                        uint8_t* q, float* scale, bool chained, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  gather_quantize_e4m3_kernel<<<(unsigned)grid_for(T), kThreads, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(x), row_of, T, k, cols, q, scale);
-  return cudaGetLastError();
+  return launch_maybe_chained(gather_quantize_e4m3_kernel, dim3((unsigned)grid_for(T)), dim3(kThreads), 0, stream,
+                              chained, static_cast<const __nv_bfloat16*>(x), row_of, T, k, cols, q, scale);
 }
 
 }  // namespace moe

@@ -19,6 +19,7 @@
 // pop the winners.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "pdl.cuh"
 
 namespace moe {
 namespace {
@@ -137,6 +138,7 @@ __global__ void __launch_bounds__(kThreads) router_topk_token_block_kernel(Route
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const T* __restrict__ x = static_cast<const T*>(p.x);
   const T* __restrict__ w = static_cast<const T*>(p.w);
+  if (threadIdx.x == 0) grid_launch_dependents();  // the dispatch may be scheduled (it waits for these ids)
   for (int64_t t = blockIdx.x; t < p.T; t += gridDim.x) {
     const T* xr = x + t * d;
     for (int e = warp; e < E; e += kWarps) {
