@@ -67,6 +67,12 @@ SMALL = {
                                             bias_select_only=1, e4m3=True, seed=34),
     "e4m3_gelu": synth.LayerConfig("e4m3_gelu", 200, 256, 16, 2, 320, "bf16", synth.SOFTMAX_ALL_RENORM, act=1,
                                    e4m3=True, seed=35),
+    # decode-sized layers whose shared expert also runs on the decode kernel:
+    # the shared GEMM-1 reuses the unit counters the routed GEMM-2 left at zero
+    "decode_shared": synth.LayerConfig("decode_shared", 24, 512, 16, 4, 256, "bf16", synth.SIGMOID_TOPK_RENORM,
+                                       n_shared=1, d_ff_shared=384, zipf_s=1.0, bias_select_only=1, seed=36),
+    "e4m3_decode_shared": synth.LayerConfig("e4m3_decode_shared", 9, 1024, 8, 2, 768, "bf16", synth.SOFTMAX_TOPK,
+                                            n_shared=1, d_ff_shared=512, e4m3=True, seed=37),
 }
 
 
@@ -94,8 +100,9 @@ def test_small_layers_full_parity(name):
     H.check_forward(inp, out)
 
 
-def test_forward_is_deterministic():
-    inp = H.make_inputs(SMALL["deepseek_like"])
+@pytest.mark.parametrize("name", ["deepseek_like", "decode_shared"])
+def test_forward_is_deterministic(name):
+    inp = H.make_inputs(SMALL[name])
     a = H.run_forward(inp)
     b = H.run_forward(inp)
     assert torch.equal(a["y"].view(torch.int16), b["y"].view(torch.int16))
