@@ -494,30 +494,60 @@ def main() -> None:
     stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
                 for j, n in enumerate(stage_names)}
 
-    # ---- end to end: pinned host x in, host y out, every step
+    # ---- end to end: pinned host x in, host y out, every step, through
+    # moe_forward.  Serving-style double buffering: step i's input copy runs
+    # on an input stream and its output copy on an output stream, so they
+    # overlap the layer of the neighbouring steps; every step's two copies lie
+    # inside the timed region (it starts before the first input copy and ends
+    # after the last output copy).
     x_host = torch.empty(T, d, dtype=tdt, pin_memory=True)
     x_host.copy_(dev["x"].cpu())
-    y_host = torch.empty(T, d, dtype=tdt, pin_memory=True)
-    x_in = torch.empty_like(dev["x"])
+    y_host = [torch.empty(T, d, dtype=tdt, pin_memory=True) for _ in range(2)]
+    x_in = [torch.empty_like(dev["x"]) for _ in range(2)]
+    y_out = [torch.empty_like(y) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("h2d", "done", "d2h")}
+    used = [False, False]
 
-    def e2e_step():
-        x_in.copy_(x_host, non_blocking=True)
-        moe.moe_forward(c, x_in, dev["w_router"], bias, dev["w_gate_up" + q], dev["w_down" + q],
-                        dev.get("ws_gate_up" + q), dev.get("ws_down" + q), y, ids, w, counts, ws, ws_bytes, stream)
-        y_host.copy_(y, non_blocking=True)
+    def e2e_step(i):
+        b = i % 2
+        if used[b]:
+            s_in.wait_event(ev["done"][b])     # x_in[b] consumed by step i - 2
+            stream.wait_event(ev["d2h"][b])    # y_out[b] copied out by step i - 2
+        with torch.cuda.stream(s_in):
+            x_in[b].copy_(x_host, non_blocking=True)
+            ev["h2d"][b].record(s_in)
+        stream.wait_event(ev["h2d"][b])
+        moe.moe_forward(c, x_in[b], dev["w_router"], bias, dev["w_gate_up" + q], dev["w_down" + q],
+                        dev.get("ws_gate_up" + q), dev.get("ws_down" + q), y_out[b], ids, w, counts, ws, ws_bytes,
+                        stream)
+        ev["done"][b].record(stream)
+        s_out.wait_event(ev["done"][b])
+        with torch.cuda.stream(s_out):
+            y_host[b].copy_(y_out[b], non_blocking=True)
+            ev["d2h"][b].record(s_out)
+        used[b] = True
 
-    for _ in range(args.warmup):
-        e2e_step()
+    for i in range(args.warmup):
+        e2e_step(i)
     torch.cuda.synchronize()
+    used[0] = used[1] = False
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+    for i in range(args.steps):
+        e2e_step(i)
+    for b in range(2):
+        if used[b]:
+            stream.wait_event(ev["d2h"][b])
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    # the last step's output, read back on the host, is the device-resident step's
+    e2e_same = bool(torch.equal(y_host[(args.steps - 1) % 2].view(torch.uint8), y.cpu().view(torch.uint8)))
 
     pk, pk_kind = peaks()
     fl = layer_flops(cfg, counts_np)
@@ -561,7 +591,9 @@ def main() -> None:
         "clocks": clocks,
         "e2e": {"value": replica_throughput(T, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * d * x_host.element_size(),
-                "d2h_bytes_per_step": T * d * y_host.element_size()},
+                "d2h_bytes_per_step": T * d * y_host[0].element_size(),
+                "copies": "pinned host <-> device every step on their own streams, double-buffered against the layer",
+                "output_matches_device_step": e2e_same},
         "gpu_launches": args.steps * launches_per_step(cfg),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
