@@ -14,15 +14,19 @@
 //   GEMM-1 (MODE_GELU, the two-matrix expert): h[rows, f] = GELU(A Wu^T).
 //   GEMM-2 (MODE_PLAIN):  y[rows, d] = h Wd^T.
 //   Router (MODE_ROUTER): logits = x W_r^T with N = E rounded up to 16; the
-//     epilogue keeps the top k per row and writes ids and gate weights.
+//     epilogue keeps the top k per row and writes ids and gate weights (one
+//     CTA per 128-token tile; see the epilogue).
 //
-// Persistent, warp-specialised CTA (192 threads, one CTA per SM):
-//   warp 0     TMA producer: 4-stage ring of (A 128x64, B Nx64) bf16 tiles,
-//              128-byte swizzle, mbarrier transaction counts
+// Persistent, warp-specialised CTA (one CTA per SM):
+//   warp 0     TMA producer: 4-stage ring of (A 128x64, B Nx64) bf16 tiles
+//              (128x128 and Nx128 with 8-bit operands), 128-byte swizzle,
+//              mbarrier transaction counts
 //   warp 1     TMEM allocator and single-thread tcgen05.mma issuer
-//              (M=128, N<=256, K=16 per instruction, fp32 accumulators)
-//   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter, SwiGLU / bf16
-//              conversion, masked 16-byte stores
+//              (M=128, N<=256, K=16 per instruction (32 for 8-bit), fp32
+//              accumulators)
+//   warps 2..  epilogue: tcgen05.ld of their 32-lane quarter, SwiGLU / bf16
+//              conversion, masked 16-byte stores; four warps in bf16, eight
+//              with 8-bit operands and in the router (kThreads)
 // Two 256-column accumulators (all 512 TMEM columns) let the epilogue of tile
 // i overlap the main loop of tile i+1.
 //
@@ -31,8 +35,9 @@
 // one expert's weight panel, so it crosses HBM about once while its row
 // blocks are still in L2.  An expert with more than 16 m-tiles (a hot expert
 // of skewed routing) is walked in blocks of 16 m-tiles, so its token rows do
-// not fall out of L2 between weight panels.  Rows past a group's end are computed on whatever
-// the TMA box holds (the next group's rows or zero fill) and never stored.
+// not fall out of L2 between weight panels.  Rows past a group's end are
+// computed on whatever the TMA box holds (the next group's rows or zero fill)
+// and never stored.
 //
 // Every wait is bounded (Params::wait_limit_ns).  On expiry the CTA raises a
 // shared abort flag and the device status word, lets its in-flight TMA loads
