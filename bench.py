@@ -98,12 +98,14 @@ def replica_throughput(tokens_per_rank: int, world: int, ms_max: float) -> float
 def launches_per_step(cfg) -> int:
     """Kernels of ours one moe_forward step launches: router, dispatch (one
     block-wide kernel for at most 1024 assignments, else count / scan /
-    scatter) and the row gather, two expert GEMMs per FFN call (routed, and
-    the shared expert's), with 8-bit experts one quantisation before each
-    GEMM, and the combine."""
+    scatter) and the row gather (with 8-bit experts the gather-quantise), two
+    expert GEMMs for the routed experts (8-bit: with the re-quantisation of h
+    between them) and for each shared expert (8-bit: after quantising x, and
+    with the re-quantisation of h), and the combine."""
     dispatch = 2 if cfg.T * cfg.top_k <= 1024 else 4
-    ffn = 2 + (2 if cfg.e4m3 else 0)
-    return 1 + dispatch + ffn * (1 + cfg.n_shared) + 1
+    routed = 2 + (1 if cfg.e4m3 else 0)
+    shared = cfg.n_shared * (2 + (2 if cfg.e4m3 else 0))
+    return 1 + dispatch + routed + shared + 1
 
 
 def peaks():
