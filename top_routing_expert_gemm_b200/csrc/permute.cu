@@ -12,7 +12,8 @@
 // Three small kernels keep the result deterministic and stable without any
 // global atomics on positions:
 //   count   : per chunk of kChunk assignments, a shared-memory histogram
-//             -> chunk_counts[e][chunk]
+//             -> chunk_counts[chunk][e] (chunk-major, so that the scan's
+//             threads, one per expert, read each chunk's row coalesced)
 //   scan    : one block turns the histograms into counts, exclusive offsets
 //             of the kept rows (min(count, C) per expert) and per-(expert,
 //             chunk) starting ranks
@@ -47,7 +48,7 @@ __global__ void __launch_bounds__(kThreads) permute_count_kernel(const int32_t* 
     else set_status(status, kDevBadExpertId);
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += kThreads) chunk_counts[(int64_t)e * n_chunks + blockIdx.x] = hist[e];
+  for (int e = threadIdx.x; e < E; e += kThreads) chunk_counts[(int64_t)blockIdx.x * E + e] = hist[e];
 }
 
 // one block of kScanThreads >= E threads
@@ -58,8 +59,17 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(int32_t* chu
   __shared__ int warp_sums[kScanThreads / 32];
   const int e = threadIdx.x, lane = e % 32, warp = e / 32;
   int total = 0;
-  if (e < E)
-    for (int b = 0; b < n_chunks; ++b) total += chunk_counts[(int64_t)e * n_chunks + b];
+  if (e < E) {  // eight independent loads in flight per thread
+    int b = 0;
+    for (; b + 8 <= n_chunks; b += 8) {
+      int c[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) c[i] = chunk_counts[(int64_t)(b + i) * E + e];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) total += c[i];
+    }
+    for (; b < n_chunks; ++b) total += chunk_counts[(int64_t)b * E + e];
+  }
   const int kept = (int)min((int64_t)total, capacity);
   // block-wide exclusive scan of the rows each expert keeps
   int incl = kept;
@@ -86,9 +96,20 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(int32_t* chu
     offsets[e] = excl;
     if (e == E - 1) offsets[E] = excl + kept;
     int run = 0;  // per-chunk starting ranks of expert e
-    for (int b = 0; b < n_chunks; ++b) {
-      const int c = chunk_counts[(int64_t)e * n_chunks + b];
-      chunk_counts[(int64_t)e * n_chunks + b] = run;
+    int b = 0;
+    for (; b + 8 <= n_chunks; b += 8) {
+      int c[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) c[i] = chunk_counts[(int64_t)(b + i) * E + e];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        chunk_counts[(int64_t)(b + i) * E + e] = run;
+        run += c[i];
+      }
+    }
+    for (; b < n_chunks; ++b) {
+      const int c = chunk_counts[(int64_t)b * E + e];
+      chunk_counts[(int64_t)b * E + e] = run;
       run += c;
     }
   }
@@ -115,7 +136,7 @@ __global__ void __launch_bounds__(kThreads) permute_scatter_kernel(const int32_t
   __syncthreads();
   // per expert: exclusive scan over the warps, starting at this chunk's base rank
   for (int e = threadIdx.x; e < E; e += kThreads) {
-    int run = chunk_base[(int64_t)e * n_chunks + blockIdx.x];
+    int run = chunk_base[(int64_t)blockIdx.x * E + e];
     for (int w = 0; w < kWarps; ++w) {
       const int c = wc[w * E + e];
       wc[w * E + e] = run;
