@@ -267,7 +267,12 @@ moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t*
 /* The whole layer: router_topk -> permute -> grouped_ffn (+ shared expert) -> combine.
    ws_gate_up [S, 2f_s, d] and ws_down [S, d, f_s] when n_shared = 1, else NULL.
    opt_topk_ids [T,k], opt_topk_w [T,k], opt_counts [E]: optional outputs (NULL = none).
-   Clears the status word first; no host synchronisation inside. */
+   Clears the status word first; no host synchronisation inside.  The kernels
+   after the router are launched with programmatic stream serialisation: each
+   may be scheduled while its predecessor finishes and waits on the device
+   before reading its predecessor's output, so stream order is kept as with
+   plain launches.  With 8-bit experts the dispatched rows are quantised while
+   they are gathered (no bf16 copy is made). */
 moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_router,
                        const float* logit_bias, const void* w_gate_up, const void* w_down,
                        const void* ws_gate_up, const void* ws_down, void* y,
