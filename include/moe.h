@@ -64,6 +64,15 @@
  *    copies, frees its tensor memory, records MOE_ERR_TIMEOUT in the status
  *    word and returns; it never traps.
  *  - Calls that share a workspace must not overlap on the GPU.
+ *  - Device: a call runs on the device that owns its workspace (moe_combine:
+ *    y; moe_quantize_e4m3: blob; moe_permute_noalloc: counts), making it
+ *    current for the duration of the call and restoring the caller's current
+ *    device before returning.  x (moe_forward) must live on that device, and
+ *    a stream created on another device is rejected (MOE_ERR_INVALID_ARG);
+ *    NULL and the legacy / per-thread default streams are the bound device's.
+ *  - Failure injection (tests): with the environment variable MOE_FAULT set to
+ *    "launch", every entry point that would launch work returns MOE_ERR_CUDA
+ *    after its host-side checks and before any CUDA call, so nothing runs.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -76,6 +85,7 @@ extern "C" {
 #endif
 
 typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
+typedef struct CUevent_st* moe_event_t;   /* identical to cudaEvent_t  */
 
 typedef enum {
   MOE_OK = 0,
@@ -185,6 +195,11 @@ moe_status moe_quantize_e4m3(const void* src, int64_t rows, int32_t cols, void* 
 int64_t moe_expert_capacity(const moe_config* cfg);
 
 /* Router + top-k + gate weights, one fused pass.
+   Defined by: "Mixture of Experts Explained: Routers, Active Parameters and
+   VRAM", the router steps Score, Normalise, Keep the top k and Renormalise;
+   "Mixture of Experts: why a model with 671 billion parameters uses only 37",
+   "The router: how a token chooses experts" and "How many experts to pick and
+   how to score them: top-k, softmax, sigmoid".
    x [T, d] (dtype), w_router [E, d] (dtype), logit_bias [E] fp32 or NULL
    -> topk_ids [T, k] int32 (slots in descending kappa), topk_w [T, k] fp32. */
 moe_status moe_router_topk(const moe_config* cfg, const void* x, const void* w_router,
@@ -212,6 +227,10 @@ moe_status moe_router_aux_losses(const moe_config* cfg, const void* x, const voi
 
 /* Dispatch: a stable counting sort of the T*k assignments by expert, then
    the row gather.
+   Defined by: "Mixture of Experts: why a model with 671 billion parameters
+   uses only 37", "How data centres handle it" (tokens grouped by their
+   assigned expert) and "Capacity factor: when tokens don't fit" (dropless
+   grouping; a capacity drops the overflow).
    topk_ids [T, k] int32, x [T, d]
    -> counts [E] (assignments routed to each expert, before any capacity cut),
       offsets [E+1] (exclusive scan of the rows each expert keeps:
@@ -238,7 +257,9 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_ids, const voi
    per-(expert, chunk) histogram lives in a 256 KiB array compiled into the
    library (held on every GPU that loads it until the process exits):
    n_experts * ceil(T*k / 2048) must be <= 65536, else MOE_ERR_UNSUPPORTED and
-   nothing runs; an invalid config returns MOE_ERR_INVALID_ARG.  The call
+   nothing runs; a config moe_permute rejects gets the same status here.  It
+   runs on the device that owns `counts` and restores the caller's current
+   device before returning (as every entry point does).  The call
    allocates nothing.  The first call on a device looks up the array's device
    address (with that device current) and keeps it for the rest of the process;
    make that first call before any stream capture, and do not reset the device
@@ -252,6 +273,12 @@ moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* topk_ids, c
                                void* x_perm, moe_stream_t stream);
 
 /* Grouped SwiGLU experts over the dispatched rows.
+   Defined by: "Mixture of Experts: why a model with 671 billion parameters
+   uses only 37", "How data centres handle it" (every expert multiply in one
+   launch over a stacked weight matrix); the expert is the "gated feed-forward
+   block with three matrices" of "Mixture of Experts Explained: Routers,
+   Active Parameters and VRAM", read as SwiGLU (or its two-matrix GELU
+   expert with MOE_ACT_GELU).
    x_perm [T*k, d], offsets [E+1] (device), w_gate_up [E, 2f, d] (rows 0..f-1
    gate, f..2f-1 up), w_down [E, d, f] -> y_perm [T*k, d].
    Rows [offsets[e], offsets[e+1]) use expert e; h [T*k, f] lives in ws. */
@@ -260,11 +287,19 @@ moe_status moe_grouped_ffn(const moe_config* cfg, const void* x_perm, const int3
                            void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Weighted un-permute: y[t] = sum_s topk_w[t,s] * y_perm[row_of[t*k+s]] (+ y_shared[t]).
+   Defined by: "Mixture of Experts Explained: Routers, Active Parameters and
+   VRAM", router step "Run and combine"; "Mixture of Experts (MoE): routing,
+   expert parallelism, and memory", "Shared experts" (the always-on add).
    y_shared [T, d] or NULL.  fp32 accumulation, y in dtype. */
 moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* row_of,
                        const float* topk_w, const void* y_shared, void* y, moe_stream_t stream);
 
 /* The whole layer: router_topk -> permute -> grouped_ffn (+ shared expert) -> combine.
+   Defined by: "Mixture of Experts: why a model with 671 billion parameters
+   uses only 37", "The router: how a token chooses experts" (the layer's
+   forward pass as a per-expert loop), computed here with grouped launches;
+   "Mixture of experts: how MoE works and what it costs", "What mixture of
+   experts means in an LLM" (routed plus shared experts).
    ws_gate_up [S, 2f_s, d] and ws_down [S, d, f_s] when n_shared = 1, else NULL.
    opt_topk_ids [T,k], opt_topk_w [T,k], opt_counts [E]: optional outputs (NULL = none).
    Clears the status word first; no host synchronisation inside.  The kernels
@@ -278,6 +313,25 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
                        const void* ws_gate_up, const void* ws_down, void* y,
                        int32_t* opt_topk_ids, float* opt_topk_w, int32_t* opt_counts,
                        void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_forward with stage markers, for per-stage timing of the layer step as
+   it runs (the pages have no counterpart; it is a tracing aid).  Same
+   arguments, checks, launches and results as moe_forward, plus
+   stage_events[6] (caller-created CUDA events; any entry, or the whole
+   array, may be NULL), each recorded on `stream` at a stage boundary:
+     [0] before the first operation of the step (the status-word clear),
+     [1] after the router, [2] after the dispatch (and the 8-bit gather),
+     [3] after the routed experts' GEMMs, [4] after the shared expert's
+     GEMMs (equal to [3] without one), [5] after the combine.
+   Elapsed time between consecutive events is that stage's device time.  A
+   recorded event separates two launches, so the next kernel of the chain
+   starts after the marker instead of overlapping its predecessor's tail. */
+moe_status moe_forward_traced(const moe_config* cfg, const void* x, const void* w_router,
+                              const float* logit_bias, const void* w_gate_up, const void* w_down,
+                              const void* ws_gate_up, const void* ws_down, void* y,
+                              int32_t* opt_topk_ids, float* opt_topk_w, int32_t* opt_counts,
+                              void* ws, size_t ws_bytes, moe_stream_t stream,
+                              const moe_event_t* stage_events);
 
 /* Synchronises `stream` and returns the status word of `ws`: MOE_OK,
    MOE_ERR_TIMEOUT or MOE_ERR_BAD_EXPERT_ID (or MOE_ERR_CUDA). */

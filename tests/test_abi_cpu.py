@@ -103,3 +103,53 @@ def test_expert_capacity_host_arithmetic(L):
     assert moe.moe_expert_capacity(_cfg(capacity_factor=float("nan"))) == -1
     assert moe.moe_expert_capacity(_cfg(expert_act=2)) == -1
     assert moe.moe_expert_capacity(_cfg(gating=4)) == -1
+
+
+def _fake(addr=256):
+    return ctypes.c_void_p(addr)
+
+
+def _launching_calls(L, cfg, ws_bytes=1 << 30):
+    """Every entry point that launches work, with valid shapes and fake aligned addresses."""
+    p, c = _fake(), ctypes.byref(cfg)
+    return {
+        "moe_router_topk": lambda: L.moe_router_topk(c, p, p, None, p, p, p, ws_bytes, None),
+        "moe_permute": lambda: L.moe_permute(c, p, p, p, p, p, p, p, p, ws_bytes, None),
+        "moe_grouped_ffn": lambda: L.moe_grouped_ffn(c, p, p, p, p, p, p, ws_bytes, None),
+        "moe_combine": lambda: L.moe_combine(c, p, p, p, None, p, None),
+        "moe_forward": lambda: L.moe_forward(c, p, p, None, p, p, None, None, p, None, None, None, p, ws_bytes,
+                                             None),
+        "moe_permute_noalloc": lambda: L.moe_permute_noalloc(c, p, p, p, p, p, p, p, None),
+        "moe_router_aux_losses": lambda: L.moe_router_aux_losses(c, p, p, p, p, p, ws_bytes, None),
+        "moe_quantize_e4m3": lambda: L.moe_quantize_e4m3(p, 64, 256, p, None),
+    }
+
+
+def test_injected_launch_failure_reports_cuda_error_after_host_checks(L, monkeypatch):
+    """MOE_FAULT=launch: each launching entry point answers MOE_ERR_CUDA once its
+    host-side checks pass (the hook sits before the first CUDA call of the
+    call, so nothing is launched; the GPU tests check that no output changes)."""
+    monkeypatch.setenv("MOE_FAULT", "launch")
+    for name, call in _launching_calls(L, _cfg()).items():
+        assert call() == 4, name
+    # host-side checks still come first: the injected failure never masks them
+    bad = _launching_calls(L, _cfg(top_k=0))
+    for name in ("moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_forward",
+                 "moe_permute_noalloc", "moe_router_aux_losses"):
+        assert bad[name]() == 1, name
+    assert _launching_calls(L, _cfg(), ws_bytes=16)["moe_forward"]() == 3
+    assert _launching_calls(L, _cfg(n_experts=2048))["moe_permute_noalloc"]() == 2
+    assert L.moe_quantize_e4m3(_fake(), 64, 250, _fake(), None) == 1
+    # any other value of the variable injects nothing
+    monkeypatch.setenv("MOE_FAULT", "none")
+    assert _launching_calls(L, _cfg(top_k=0))["moe_forward"]() == 1
+
+
+def test_noalloc_dispatch_reports_the_same_config_status_as_moe_permute(L):
+    for cfg, want in ((_cfg(n_experts=2048), 2), (_cfg(top_k=17, n_experts=32), 2), (_cfg(top_k=0), 1),
+                      (_cfg(d_model=250), 1), (_cfg(n_shared=2, d_ff_shared=512), 2)):
+        got = L.moe_permute_noalloc(ctypes.byref(cfg), _fake(), _fake(), _fake(), _fake(), _fake(), _fake(),
+                                    _fake(), None)
+        ref = L.moe_permute(ctypes.byref(cfg), _fake(), _fake(), _fake(), _fake(), _fake(), _fake(), _fake(),
+                            _fake(), 1 << 30, None)
+        assert got == ref == want, (cfg.n_experts, cfg.top_k, got, ref)

@@ -36,3 +36,50 @@ def test_expired_wait_limit_reports_timeout_and_context_survives(cfg):
     good = H.run_forward(inp)
     assert good["status"] == 0
     H.check_forward(inp, good)
+
+
+def test_injected_launch_failure_launches_nothing_and_the_next_call_runs(monkeypatch):
+    """MOE_FAULT=launch (a host-side hook; nothing is injected on the device):
+    every launching entry point reports MOE_ERR_CUDA, its outputs keep their
+    canary values and the workspace status word is untouched; with the
+    variable cleared the same call runs and matches the oracle."""
+    cfg = synth.workload("tiny_f32").replace(T=64, seed=31)
+    inp = H.make_inputs(cfg)
+    c = H.moe_cfg(cfg)
+    dev = inp.dev
+    T, k, E, d = cfg.T, cfg.top_k, cfg.n_experts, cfg.d_model
+    ws = torch.full((moe.moe_workspace_bytes(c),), 0x5A, dtype=torch.uint8, device="cuda")
+    y = torch.full((T, d), 7.0, dtype=torch.float32, device="cuda")
+    ids = torch.full((T, k), -9, dtype=torch.int32, device="cuda")
+    w = torch.full((T, k), 3.0, dtype=torch.float32, device="cuda")
+    counts = torch.full((E,), -9, dtype=torch.int32, device="cuda")
+    offsets = torch.full((E + 1,), -9, dtype=torch.int32, device="cuda")
+    perm = torch.full((T * k,), -9, dtype=torch.int32, device="cuda")
+    row_of = torch.full((T * k,), -9, dtype=torch.int32, device="cuda")
+    x_perm = torch.full((T * k, d), 5.0, dtype=torch.float32, device="cuda")
+    canaries = [t.clone() for t in (ws, y, ids, w, counts, offsets, perm, row_of, x_perm)]
+    ids_in = torch.zeros(T, k, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    calls = {
+        "moe_forward": lambda: moe.moe_forward(c, dev["x"], dev["w_router"], None, dev["w_gate_up"], dev["w_down"],
+                                               None, None, y, ids, w, counts, ws),
+        "moe_router_topk": lambda: moe.moe_router_topk(c, dev["x"], dev["w_router"], None, ids, w, ws),
+        "moe_permute": lambda: moe.moe_permute(c, ids_in, dev["x"], counts, offsets, perm, row_of, x_perm, ws),
+        "moe_permute_noalloc": lambda: moe.moe_permute_noalloc(c, ids_in, dev["x"], counts, offsets, perm, row_of,
+                                                               x_perm),
+        "moe_grouped_ffn": lambda: moe.moe_grouped_ffn(c, x_perm, offsets, dev["w_gate_up"], dev["w_down"], x_perm,
+                                                       ws),
+        "moe_combine": lambda: moe.moe_combine(c, x_perm, row_of, w, None, y),
+    }
+    monkeypatch.setenv("MOE_FAULT", "launch")
+    for name, call in calls.items():
+        with pytest.raises(moe.MoeError) as e:
+            call()
+        assert e.value.status == 4, name
+    torch.cuda.synchronize()
+    for before, after in zip(canaries, (ws, y, ids, w, counts, offsets, perm, row_of, x_perm)):
+        assert torch.equal(before, after)
+    monkeypatch.delenv("MOE_FAULT")
+    good = H.run_forward(inp)
+    assert good["status"] == 0
+    H.check_forward(inp, good)

@@ -14,7 +14,7 @@ __all__ = [
     "MoeError", "MoeConfig", "lib", "make_config", "moe_workspace_bytes", "moe_status_string",
     "moe_router_topk", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_forward", "moe_device_status",
     "moe_permute_noalloc", "moe_expert_capacity", "moe_router_aux_losses", "moe_e4m3_weight_bytes",
-    "moe_quantize_e4m3", "MOE_W_NATIVE", "MOE_W_E4M3",
+    "moe_quantize_e4m3", "moe_forward_traced", "MOE_W_NATIVE", "MOE_W_E4M3",
     "MOE_F32", "MOE_BF16", "MOE_SOFTMAX_ALL_RENORM", "MOE_SOFTMAX_TOPK", "MOE_SIGMOID_TOPK_RENORM",
     "MOE_SOFTMAX_ALL_NO_RENORM", "MOE_ACT_SWIGLU", "MOE_ACT_GELU",
     "EXPORTED_SYMBOLS", "LIB_PATH",
@@ -33,7 +33,7 @@ MOE_W_NATIVE, MOE_W_E4M3 = 0, 1
 EXPORTED_SYMBOLS = (
     "moe_workspace_bytes", "moe_status_string", "moe_router_topk", "moe_permute", "moe_grouped_ffn",
     "moe_combine", "moe_forward", "moe_device_status", "moe_permute_noalloc", "moe_expert_capacity",
-    "moe_router_aux_losses", "moe_e4m3_weight_bytes", "moe_quantize_e4m3",
+    "moe_router_aux_losses", "moe_e4m3_weight_bytes", "moe_quantize_e4m3", "moe_forward_traced",
 )
 
 
@@ -83,6 +83,8 @@ def lib() -> ctypes.CDLL:
         L.moe_grouped_ffn.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_combine.argtypes = [cfgp, vp, vp, vp, vp, vp, vp]
         L.moe_forward.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_forward_traced.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
+                                         ctypes.POINTER(vp)]
         L.moe_device_status.argtypes = [vp, sz, vp]
         L.moe_permute_noalloc.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.moe_expert_capacity.argtypes = [cfgp]
@@ -192,6 +194,41 @@ def moe_forward(cfg, x, w_router, logit_bias, w_gate_up, w_down, ws_gate_up, ws_
     _check(lib().moe_forward(ctypes.byref(cfg), _p(x), _p(w_router), _p(logit_bias), _p(w_gate_up), _p(w_down),
                              _p(ws_gate_up), _p(ws_down), _p(y), _p(opt_topk_ids), _p(opt_topk_w),
                              _p(opt_counts), _p(ws), nb, _stream(stream)), "moe_forward")
+
+
+def moe_forward_traced(cfg, x, w_router, logit_bias, w_gate_up, w_down, ws_gate_up, ws_down, y,
+                       opt_topk_ids=None, opt_topk_w=None, opt_counts=None, ws=None, ws_bytes=None, stream=None,
+                       stage_events=None) -> None:
+    """moe_forward with six stage markers: ``stage_events`` is a sequence of six
+    torch.cuda.Event (or None entries) recorded at the stage boundaries."""
+    nb = ws_bytes if ws_bytes is not None else ws.numel() * ws.element_size()
+    arr = None
+    if stage_events is not None:
+        if len(stage_events) != 6:
+            raise ValueError("stage_events needs six entries")
+        handles = []
+        for ev in stage_events:
+            if ev is None:
+                handles.append(None)
+                continue
+            if not ev.cuda_event:  # torch creates its events on the first record
+                ev.record(torch_stream(stream))
+            handles.append(ev.cuda_event)
+        arr = (ctypes.c_void_p * 6)(*handles)
+    _check(lib().moe_forward_traced(ctypes.byref(cfg), _p(x), _p(w_router), _p(logit_bias), _p(w_gate_up),
+                                    _p(w_down), _p(ws_gate_up), _p(ws_down), _p(y), _p(opt_topk_ids),
+                                    _p(opt_topk_w), _p(opt_counts), _p(ws), nb, _stream(stream), arr),
+           "moe_forward_traced")
+
+
+def torch_stream(stream):
+    """The torch stream object for the ``stream`` argument of the calls above."""
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream()
+    if isinstance(stream, int):
+        return torch.cuda.ExternalStream(stream)
+    return stream
 
 
 def moe_device_status(ws, ws_bytes=None, stream=None) -> int:

@@ -8,6 +8,7 @@
 
 #include "../../include/moe.h"
 #include "common.cuh"
+#include "host_guard.cuh"
 #include "kernels.cuh"
 
 namespace moe {
@@ -29,13 +30,6 @@ cudaError_t launch_router_topk(const RouterArgs& a, cudaStream_t stream) {
   if (router_uses_tc(a.bf16, a.E, a.T)) return launch_router_topk_tc(a, stream);
   return launch_router_topk_simt(a, stream);
 }
-
-namespace {
-
-constexpr size_t kAlign = 256;
-inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 moe_status check_config(const moe_config* c) {
   if (c == nullptr) return MOE_ERR_INVALID_ARG;
@@ -64,6 +58,13 @@ moe_status check_config(const moe_config* c) {
     return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 size_t elem_bytes(const moe_config* c) { return c->dtype == MOE_BF16 ? 2 : 4; }
 
@@ -158,28 +159,15 @@ moe_status check_ws(const moe_config* c, const void* ws, size_t ws_bytes) {
   return MOE_OK;
 }
 
-// Make the runtime's current device the one that owns `p`; rejects host pointers.
-cudaError_t bind_device(const void* p) {
-  cudaPointerAttributes at;
-  cudaError_t e = cudaPointerGetAttributes(&at, p);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return e;
-  }
-  if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged) return cudaErrorInvalidValue;
-  int cur = -1;
-  e = cudaGetDevice(&cur);
-  if (e != cudaSuccess) return e;
-  return cur == at.device ? cudaSuccess : cudaSetDevice(at.device);
-}
-
-moe_status bind(const void* p) {
-  const cudaError_t e = bind_device(p);
-  if (e == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;
-  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
-}
-
 uint64_t wait_limit(const moe_config* c) { return c->wait_limit_ns > 0 ? (uint64_t)c->wait_limit_ns : 2000000000ull; }
+
+// After a call's host checks: the injected launch failure (host_guard.cuh),
+// then the switch to the device that owns `p` and the check of the stream.
+moe_status enter(DeviceGuard& g, const void* p, cudaStream_t stream) {
+  if (launch_failure_injected()) return MOE_ERR_CUDA;
+  const moe_status st = g.bind(p);
+  return st != MOE_OK ? st : g.check_stream(stream);
+}
 
 // a_quantized: 8-bit experts whose input rows are already in xq / sx;
 // chained: a layer step that cleared the decode counters ahead and chains its
@@ -231,8 +219,9 @@ moe_status moe_quantize_e4m3(const void* src, int64_t rows, int32_t cols, void* 
   if (rows == 0) return MOE_OK;
   if (!src || !blob || !aligned16(src) || (reinterpret_cast<uintptr_t>(blob) % kAlign) != 0)
     return MOE_ERR_INVALID_ARG;
-  moe_status st;
-  if ((st = bind(blob)) != MOE_OK) return st;
+  DeviceGuard g;
+  const moe_status st = enter(g, blob, stream);
+  if (st != MOE_OK) return st;
   uint8_t* q = static_cast<uint8_t*>(blob);
   float* sc = reinterpret_cast<float*>(q + e4m3_codes_bytes(rows, cols));
   MOE_CUDA_TRY(launch_quantize_e4m3(src, rows, nullptr, cols, q, sc, stream));
@@ -266,7 +255,8 @@ moe_status moe_router_topk(const moe_config* cfg, const void* x, const void* w_r
   if (!x || !w_router || !topk_ids || !topk_w || !aligned16(x) || !aligned16(w_router) || !aligned16(topk_ids) ||
       !aligned16(topk_w) || (logit_bias && !aligned16(logit_bias)))
     return MOE_ERR_INVALID_ARG;
-  if ((st = bind(ws)) != MOE_OK) return st;
+  DeviceGuard g;
+  if ((st = enter(g, ws, stream)) != MOE_OK) return st;
   Carve k = carve(cfg, ws);
   RouterArgs a{x, w_router, logit_bias, topk_ids, topk_w, cfg->T, cfg->d_model, cfg->n_experts, cfg->top_k,
                cfg->gating, cfg->bias_select_only, cfg->dtype == MOE_BF16, k.status, wait_limit(cfg)};
@@ -281,7 +271,8 @@ moe_status moe_router_aux_losses(const moe_config* cfg, const void* x, const voi
   if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
   if (!counts || !out || !aligned16(counts) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
   if (cfg->T > 0 && (!x || !w_router || !aligned16(x) || !aligned16(w_router))) return MOE_ERR_INVALID_ARG;
-  if ((st = bind(ws)) != MOE_OK) return st;
+  DeviceGuard g;
+  if ((st = enter(g, ws, stream)) != MOE_OK) return st;
   if (cfg->T == 0) {
     MOE_CUDA_TRY(cudaMemsetAsync(out, 0, 2 * sizeof(float), stream));
     return MOE_OK;
@@ -304,7 +295,8 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_ids, const voi
   if (cfg->T > 0 && (!topk_ids || !perm || !row_of || !x || !x_perm || !aligned16(topk_ids) || !aligned16(perm) ||
                      !aligned16(row_of) || !aligned16(x) || !aligned16(x_perm)))
     return MOE_ERR_INVALID_ARG;
-  if ((st = bind(ws)) != MOE_OK) return st;
+  DeviceGuard g;
+  if ((st = enter(g, ws, stream)) != MOE_OK) return st;
   Carve k = carve(cfg, ws);
   PermuteArgs a{topk_ids, x, counts, offsets, perm, row_of, x_perm, k.chunk_counts, cfg->T * cfg->top_k,
                 cfg->top_k, cfg->d_model, cfg->n_experts, (int)elem_bytes(cfg), k.status, capacity_rows(cfg)};
@@ -321,7 +313,8 @@ moe_status moe_grouped_ffn(const moe_config* cfg, const void* x_perm, const int3
   if (!x_perm || !offsets || !w_gate_up || !w_down || !y_perm || !aligned16(x_perm) || !aligned16(offsets) ||
       !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(y_perm))
     return MOE_ERR_INVALID_ARG;
-  if ((st = bind(ws)) != MOE_OK) return st;
+  DeviceGuard g;
+  if ((st = enter(g, ws, stream)) != MOE_OK) return st;
   Carve k = carve(cfg, ws);
   MOE_CUDA_TRY(run_ffn(cfg, k, x_perm, offsets, cfg->n_experts, cfg->T * cfg->top_k, cfg->d_ff, w_gate_up, w_down,
                        k.h, y_perm, stream));
@@ -336,7 +329,8 @@ moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t*
   if (!y_perm || !row_of || !topk_w || !y || !aligned16(y_perm) || !aligned16(row_of) || !aligned16(topk_w) ||
       !aligned16(y) || (y_shared && !aligned16(y_shared)))
     return MOE_ERR_INVALID_ARG;
-  if ((st = bind(y)) != MOE_OK) return st;
+  DeviceGuard g;
+  if ((st = enter(g, y, stream)) != MOE_OK) return st;
   CombineArgs a{y_perm, row_of, topk_w, y_shared, y, cfg->T, cfg->top_k, cfg->d_model, cfg->dtype == MOE_BF16};
   MOE_CUDA_TRY(launch_combine(a, stream));
   return MOE_OK;
@@ -346,12 +340,27 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
                        const void* w_gate_up, const void* w_down, const void* ws_gate_up, const void* ws_down,
                        void* y, int32_t* opt_topk_ids, float* opt_topk_w, int32_t* opt_counts, void* ws,
                        size_t ws_bytes, moe_stream_t stream) {
+  return moe_forward_traced(cfg, x, w_router, logit_bias, w_gate_up, w_down, ws_gate_up, ws_down, y, opt_topk_ids,
+                            opt_topk_w, opt_counts, ws, ws_bytes, stream, nullptr);
+}
+
+moe_status moe_forward_traced(const moe_config* cfg, const void* x, const void* w_router, const float* logit_bias,
+                              const void* w_gate_up, const void* w_down, const void* ws_gate_up,
+                              const void* ws_down, void* y, int32_t* opt_topk_ids, float* opt_topk_w,
+                              int32_t* opt_counts, void* ws, size_t ws_bytes, moe_stream_t stream,
+                              const moe_event_t* stage_events) {
+  // stage boundary i: record stage_events[i] (when given) on the stream
+  auto mark = [&](int i) -> cudaError_t {
+    if (stage_events == nullptr || stage_events[i] == nullptr) return cudaSuccess;
+    return cudaEventRecord(stage_events[i], stream);
+  };
   moe_status st = check_config(cfg);
   if (st != MOE_OK) return st;
   if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
   if (cfg->T == 0) {  // nothing to read or write: clear the status word and the optional counts
     if (opt_counts && !aligned16(opt_counts)) return MOE_ERR_INVALID_ARG;
-    if ((st = bind(ws)) != MOE_OK) return st;
+    DeviceGuard g;
+    if ((st = enter(g, ws, stream)) != MOE_OK) return st;
     MOE_CUDA_TRY(cudaMemsetAsync(ws, 0, 16, stream));
     if (opt_counts) MOE_CUDA_TRY(cudaMemsetAsync(opt_counts, 0, sizeof(int32_t) * cfg->n_experts, stream));
     return MOE_OK;
@@ -363,9 +372,11 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
     return MOE_ERR_INVALID_ARG;
   if (cfg->n_shared > 0 && (!ws_gate_up || !ws_down || !aligned16(ws_gate_up) || !aligned16(ws_down)))
     return MOE_ERR_INVALID_ARG;
-  if ((st = bind(ws)) != MOE_OK) return st;
-  if ((st = bind(x)) != MOE_OK) return st;
+  DeviceGuard g;
+  if ((st = enter(g, ws, stream)) != MOE_OK) return st;
+  if ((st = g.same_device(x)) != MOE_OK) return st;
   Carve k = carve(cfg, ws);
+  MOE_CUDA_TRY(mark(0));
   MOE_CUDA_TRY(cudaMemsetAsync(k.status, 0, 16, stream));
   // The launches of the step are chained (pdl.cuh): each kernel after the
   // router may be scheduled while its predecessor finishes.  The decode
@@ -378,6 +389,7 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
   RouterArgs ra{x, w_router, logit_bias, ids, w, cfg->T, cfg->d_model, cfg->n_experts, cfg->top_k,
                 cfg->gating, cfg->bias_select_only, cfg->dtype == MOE_BF16, k.status, wait_limit(cfg)};
   MOE_CUDA_TRY(launch_router_topk(ra, stream));
+  MOE_CUDA_TRY(mark(1));
   // 8-bit experts: the dispatch writes no bf16 copy; each token is quantised
   // once, straight from x, and its codes go to its rows
   const bool e4m3 = cfg->weight_format == MOE_W_E4M3;
@@ -388,14 +400,18 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
   if (e4m3)
     MOE_CUDA_TRY(
         launch_gather_quantize_e4m3(x, k.row_of, cfg->top_k, cfg->T, cfg->d_model, k.xq, k.sx, true, stream));
+  MOE_CUDA_TRY(mark(2));
   MOE_CUDA_TRY(run_ffn(cfg, k, k.x_perm, k.offsets, cfg->n_experts, cfg->T * cfg->top_k, cfg->d_ff, w_gate_up,
                        w_down, k.h, k.y_perm, stream, false, e4m3, true));
+  MOE_CUDA_TRY(mark(3));
   if (cfg->n_shared > 0)
     MOE_CUDA_TRY(run_ffn(cfg, k, x, nullptr, 1, cfg->T, cfg->d_ff_shared, ws_gate_up, ws_down, k.h_s, k.y_s, stream,
                          true, false, true));
+  MOE_CUDA_TRY(mark(4));
   CombineArgs ca{k.y_perm, k.row_of, w, cfg->n_shared > 0 ? k.y_s : nullptr, y, cfg->T, cfg->top_k,
                  cfg->d_model, cfg->dtype == MOE_BF16, true};
   MOE_CUDA_TRY(launch_combine(ca, stream));
+  MOE_CUDA_TRY(mark(5));
   return MOE_OK;
 }
 

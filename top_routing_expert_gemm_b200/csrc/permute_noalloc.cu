@@ -15,6 +15,7 @@
 
 #include "../../include/moe.h"
 #include "common.cuh"
+#include "host_guard.cuh"
 #include "kernels.cuh"
 
 namespace moe {
@@ -57,7 +58,8 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
                                           int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* row_of,
                                           void* x_perm, moe_stream_t stream) {
   using namespace moe;
-  if (moe_workspace_bytes(cfg) == 0) return MOE_ERR_INVALID_ARG;  // config check only, allocates nothing
+  moe_status st = check_config(cfg);  // the same statuses as moe_permute; allocates nothing
+  if (st != MOE_OK) return st;
   const int64_t n = cfg->T * cfg->top_k;
   const int64_t need = (int64_t)cfg->n_experts * permute_n_chunks(n);
   if (need > kNoAllocScratchInts) return MOE_ERR_UNSUPPORTED;
@@ -65,16 +67,12 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
   if (cfg->T > 0 && (!topk_ids || !perm || !row_of || !x || !x_perm || !aligned16(topk_ids) || !aligned16(perm) ||
                      !aligned16(row_of) || !aligned16(x) || !aligned16(x_perm)))
     return MOE_ERR_INVALID_ARG;
-  // run on the device that owns the outputs
-  cudaPointerAttributes at;
-  if (cudaPointerGetAttributes(&at, counts) != cudaSuccess) {
-    cudaGetLastError();
-    return MOE_ERR_INVALID_ARG;
-  }
-  if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged) return MOE_ERR_INVALID_ARG;
-  int cur = -1;
-  if (cudaGetDevice(&cur) != cudaSuccess) return MOE_ERR_CUDA;
-  if (cur != at.device && cudaSetDevice(at.device) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_failure_injected()) return MOE_ERR_CUDA;
+  // run on the device that owns the outputs; the caller's current device is
+  // restored when the guard goes out of scope
+  DeviceGuard g;
+  if ((st = g.bind(counts)) != MOE_OK) return st;
+  if ((st = g.check_stream(stream)) != MOE_OK) return st;
   int32_t* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
   // The histogram pass writes every (expert, chunk) entry this call later
