@@ -9,20 +9,23 @@ Generator
 ---------
 Every tensor is a pure function of ``(seed, stream, flat element index)``:
 
-* a 32-bit counter hash built from the MurmurHash3 ``fmix32`` finaliser,
-  applied twice (low word of the index, then high word), once per "lane";
-* two lanes give four 16-bit uniform integers ``u0..u3``;
-* an approximately standard normal value is their standardised
-  Irwin-Hall sum ``z = ((u0+u1+u2+u3+2)/65536 - 2) * sqrt(3)``
-  (mean 0, variance 1, support +-2*sqrt(3));
+* a 32-bit counter hash U built from the MurmurHash3 ``fmix32`` finaliser,
+  applied twice (low word of the index, then high word);
+* a standard normal value by the inverse-CDF method: U picks one of 2**20
+  equal-probability cells (its top 20 bits) and a point inside it (its low 12
+  bits, offset by half a step); the value interpolates linearly between the
+  normal quantiles at the cell's edges, ``Phi^-1(j / 2**20)``, taken from a
+  table computed once in float64 (the two outermost edges are clamped at
+  ``Phi^-1(2**-33)``, about -6.1 and +6.1);
 * ``value = float32(z * std)`` with ``std = 1/sqrt(fan_in)`` for weights and
   1 for activations, then rounded to bfloat16 (round-to-nearest-even) for the
   bf16 workloads.
 
-Only integer operations and correctly rounded IEEE-754 binary64 ``+ - * /``
-appear, so the numpy (host) and torch (device) implementations below return
-bit-identical values; any element can be regenerated on its own, which lets
-the oracle rebuild exactly the slices it needs.
+Only integer operations, a table lookup and correctly rounded IEEE-754
+binary64 ``+ - * /`` (each a separate operation, no fused multiply-add)
+appear per element, so the numpy (host) and torch (device) implementations
+below return bit-identical values; any element can be regenerated on its
+own, which lets the oracle rebuild exactly the slices it needs.
 
 Streams: x=0, router=1, routed gate/up=2, routed down=3, shared gate/up=4,
 shared down=5, routing-bias permutation=6.  Seed = 1000 + workload index.
@@ -35,7 +38,6 @@ import math
 import numpy as np
 
 MASK32 = 0xFFFFFFFF
-SQRT3 = math.sqrt(3.0)
 
 STREAM_X = 0
 STREAM_ROUTER = 1
@@ -98,10 +100,39 @@ def _hash_lane(idx, seed: int, stream: int, lane: int):
     return h
 
 
-def _irwin_hall_sum(idx, seed: int, stream: int):
-    h0 = _hash_lane(idx, seed, stream, 0)
-    h1 = _hash_lane(idx, seed, stream, 1)
-    return (h0 & 0xFFFF) + (h0 >> 16) + (h1 & 0xFFFF) + (h1 >> 16)
+QUANTILE_BITS = 20          # 2**20 equal-probability cells
+FRAC_BITS = 32 - QUANTILE_BITS
+_TABLE = {}
+
+
+def quantile_table() -> np.ndarray:
+    """Normal quantiles at the 2**20 + 1 cell edges j / 2**20 (float64); the
+    infinite outer edges are clamped at Phi^-1(2**-33) and its negative."""
+    if "host" not in _TABLE:
+        from scipy.special import ndtri
+
+        m = 1 << QUANTILE_BITS
+        q = ndtri(np.arange(m + 1, dtype=np.float64) / m)
+        q[0] = ndtri(2.0 ** -33)
+        q[m] = -q[0]
+        _TABLE["host"] = q
+    return _TABLE["host"]
+
+
+def _device_table(device):
+    import torch
+
+    key = str(device)
+    if key not in _TABLE:
+        _TABLE[key] = torch.from_numpy(quantile_table()).to(device)
+    return _TABLE[key]
+
+
+def _cell_and_fraction(idx, seed: int, stream: int):
+    """Cell index (top 20 bits of the hash) and the point inside the cell,
+    ((low 12 bits) + 0.5) / 2**12 as an exact binary64 fraction."""
+    u = _hash_lane(idx, seed, stream, 0)
+    return u >> FRAC_BITS, u & ((1 << FRAC_BITS) - 1)
 
 
 # --------------------------------------------------------------------------
@@ -110,8 +141,11 @@ def _irwin_hall_sum(idx, seed: int, stream: int):
 def normal_f32(seed: int, stream: int, start: int, count: int, std: float = 1.0) -> np.ndarray:
     """float32 values of elements [start, start+count) of one stream (numpy)."""
     idx = np.arange(start, start + count, dtype=np.int64)
-    s = _irwin_hall_sum(idx, seed, stream)
-    z = ((s + 2).astype(np.float64) / 65536.0 - 2.0) * SQRT3
+    j, lo = _cell_and_fraction(idx, seed, stream)
+    q = quantile_table()
+    q0, q1 = q[j], q[j + 1]
+    f = (lo.astype(np.float64) + 0.5) / float(1 << FRAC_BITS)
+    z = q0 + f * (q1 - q0)
     if std != 1.0:
         z = z * np.float64(std)
     return z.astype(np.float32)
@@ -151,10 +185,17 @@ def normal_torch(seed: int, stream: int, start: int, count: int, std: float, dty
     for c0 in range(0, count, chunk):
         n = min(chunk, count - c0)
         idx = torch.arange(start + c0, start + c0 + n, dtype=torch.int64, device=device)
-        s = _irwin_hall_sum(idx, seed, stream)
+        j, lo = _cell_and_fraction(idx, seed, stream)
         del idx
-        z = ((s + 2).to(torch.float64) / 65536.0 - 2.0) * SQRT3
-        del s
+        q = _device_table(device)
+        q0, q1 = q[j], q[j + 1]
+        del j
+        f = (lo.to(torch.float64) + 0.5) / float(1 << FRAC_BITS)
+        del lo
+        d = q1 - q0
+        del q1
+        z = q0 + f * d
+        del q0, d, f
         if std != 1.0:
             z = z * std
         flat[c0:c0 + n] = z.to(torch.float32).to(tdt)

@@ -26,14 +26,27 @@ def test_bf16_rounding_is_nearest_even():
     assert synth.bf16_bits_to_f32(ours)[2] == 1.0 + 2 ** -6  # tie rounds up to even
 
 
-def test_moments_and_support():
-    v = synth.normal_f32(7, 0, 0, 1 << 20).astype(np.float64)
-    assert abs(v.mean()) < 5e-3
-    assert abs(v.var() - 1.0) < 5e-3
-    assert np.max(np.abs(v)) <= 2 * math.sqrt(3.0)
-    # excess kurtosis of the 4-term Irwin-Hall sum is -0.3
-    k = np.mean(v ** 4) / v.var() ** 2 - 3.0
-    assert abs(k + 0.3) < 0.02
+def test_moments_support_and_quantiles_are_standard_normal():
+    v = synth.normal_f32(7, 0, 0, 1 << 22).astype(np.float64)
+    n = len(v)
+    assert abs(v.mean()) < 4.0 / math.sqrt(n)
+    assert abs(v.var() - 1.0) < 5.0 * math.sqrt(2.0 / n)
+    assert np.max(np.abs(v)) <= 6.2
+    k = np.mean(v ** 4) / v.var() ** 2 - 3.0          # excess kurtosis of a normal is 0
+    assert abs(k) < 0.02
+    # tail probabilities of N(0,1): P(z < -1.96) = 0.025, P(z < -3) = 0.00135, P(z > 4) = 3.2e-5
+    for z, p in ((-1.959963984540054, 0.025), (-3.0, 0.0013498980316301), (-4.0, 3.167124183311998e-05)):
+        got = np.mean(v < z)
+        assert abs(got - p) < 5.0 * math.sqrt(p * (1 - p) / n) + 1e-6, (z, got, p)
+
+
+def test_quantile_table_edges_are_normal_quantiles():
+    q = synth.quantile_table()
+    m = 1 << synth.QUANTILE_BITS
+    assert len(q) == m + 1 and np.all(np.diff(q) > 0)
+    assert q[m // 2] == 0.0
+    assert abs(q[int(0.975 * m)] - 1.959963984540054) < 1e-5   # Phi^-1(0.975)
+    assert np.allclose(q[1:m][::-1], -q[1:m], rtol=0, atol=1e-9)
 
 
 def test_slices_regenerate_the_whole():
