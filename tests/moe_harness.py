@@ -197,6 +197,43 @@ def sample_tokens(T: int, n: int, seed: int = 0) -> np.ndarray:
     return np.sort(np.concatenate([[0, T - 1], mid]))
 
 
+TILE_ROWS = 128          # token rows per tile of the large-batch expert GEMMs
+BLOCK_ROWS = 16 * 128    # rows of one block of a hot expert's walk (16 m-tiles)
+
+
+def coverage_tokens(offsets: np.ndarray, perm: np.ndarray, k: int, T: int, n_min: int,
+                    seed: int = 0) -> np.ndarray:
+    """Tokens whose rows reach the parts of the grouped GEMMs that only full
+    sizes exercise: every expert's last row and the first row of its last
+    (partial) 128-row tile, the rows on both sides of every 2048-row block
+    boundary of the hottest expert, the first and last dispatched rows (the
+    experts after the persistent grid's first wave are among "every expert");
+    then random tokens up to ``n_min``.  ``offsets``/``perm`` are the dispatch
+    of the routing under test."""
+    want = set()
+    E = len(offsets) - 1
+    n = np.diff(offsets)
+    for e in range(E):
+        if n[e] <= 0:
+            continue
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        want.add(int(perm[hi - 1]) // k)
+        want.add(int(perm[lo + ((hi - lo - 1) // TILE_ROWS) * TILE_ROWS]) // k)
+    hot = int(np.argmax(n))
+    for b in range(BLOCK_ROWS, int(n[hot]), BLOCK_ROWS):
+        for r in (b - 1, b):
+            want.add(int(perm[offsets[hot] + r]) // k)
+    if offsets[-1] > 0:
+        want.add(int(perm[0]) // k)
+        want.add(int(perm[offsets[-1] - 1]) // k)
+    rng = np.random.default_rng(seed)
+    rest = np.setdiff1d(np.arange(T), np.fromiter(want, dtype=np.int64))
+    extra = max(0, n_min - len(want))
+    if extra and len(rest):
+        want |= set(rng.choice(rest, size=min(extra, len(rest)), replace=False).tolist())
+    return np.array(sorted(want), dtype=np.int64)
+
+
 def check_forward(inp: Inputs, out: dict, n_sample: int | None = None) -> dict:
     """Parity of one moe_forward call against the oracle.
 
@@ -218,10 +255,10 @@ def check_forward(inp: Inputs, out: dict, n_sample: int | None = None) -> dict:
     r = oracle.route(x_all, wr, bias, k, cfg.gating, cfg.bias_select_only)
     stats = check_routing(cfg, gpu_ids, gpu_w, r, T)
     cap = capacity_of(cfg)
-    counts, _offsets, _perm, row_of = oracle.dispatch(gpu_ids, E, cap)
+    counts, offsets, perm, row_of = oracle.dispatch(gpu_ids, E, cap)
     assert np.array_equal(out["counts"].cpu().numpy(), counts)
     keep = (row_of >= 0).reshape(T, k)  # slots the capacity keeps, decided over the whole batch
-    tokens = np.arange(T) if n_sample is None else sample_tokens(T, n_sample)
+    tokens = np.arange(T) if n_sample is None else coverage_tokens(offsets, perm, k, T, n_sample)
     y_ref, _, _ = oracle.moe_layer(x_all[tokens], wr, bias, k, cfg.gating, ow.routed, E,
                                    shared_weights=ow.shared(), bias_select_only=cfg.bias_select_only,
                                    ids=gpu_ids[tokens], act=cfg.act, keep=keep[tokens], e4m3=cfg.e4m3)

@@ -64,3 +64,47 @@ def test_launches_per_step():
     # routed GEMMs, the shared expert's x and h quantised
     assert bench.launches_per_step(synth.workload("mixtral_bf16", e4m3=True)) == 9
     assert bench.launches_per_step(synth.workload("deepseek_bf16", e4m3=True)) == 13
+
+
+def test_workload_keys_and_selection():
+    assert bench.workload_key("decode_bf16", {"T": 4}) == "decode_bf16[T=4]"
+    assert bench.workload_key("decode_bf16", {"T": 16, "zipf_s": 1.2}) == "decode_bf16[T=16,zipf=1.2]"
+    assert bench.workload_key("gptoss_bf16", {"e4m3": True}) == "gptoss_bf16[e4m3]"
+    keys = [bench.workload_key(n, ov) for n, ov in bench.parse_workloads("all", "mixtral_bf16")]
+    assert len(keys) == len(set(keys)) == len(bench.EXTRA_WORKLOADS)
+    assert {"gptoss_bf16", "deepseek_bf16", "tiny_f32", "decode_bf16[T=1]", "decode_bf16[T=64,zipf=1.2]",
+            "mixtral_bf16[e4m3]"} <= set(keys)
+    assert bench.parse_workloads("none", "mixtral_bf16") == []
+    assert [bench.workload_key(n, ov) for n, ov in bench.parse_workloads("decode_bf16[T=4],tiny_f32", "x")] == \
+        ["decode_bf16[T=4]", "tiny_f32"]
+
+
+def test_l2_flush_only_for_inputs_that_fit_in_l2():
+    assert bench.needs_l2_flush(synth.workload("tiny_f32"))
+    for name in ("mixtral_bf16", "gptoss_bf16", "deepseek_bf16"):
+        assert not bench.needs_l2_flush(synth.workload(name))
+    assert not bench.needs_l2_flush(synth.workload("decode_bf16", T=1))
+
+
+def test_oracle_sample_is_the_batch_or_a_fixed_subset():
+    assert bench.oracle_sample_tokens(synth.workload("mixtral_bf16")) == 2048
+    assert bench.oracle_sample_tokens(synth.workload("tiny_f32")) == 256
+    assert bench.oracle_sample_tokens(synth.workload("gptoss_bf16")) == 1024
+    assert bench.oracle_sample_tokens(synth.workload("decode_bf16", T=4)) == 4
+
+
+def test_roofline_of_follows_from_its_numbers():
+    cfg = synth.workload("mixtral_bf16")
+    counts = np.array([512] * 8)
+    stage = {"routed_ffn": 1.0, "shared_ffn": 0.0}
+    pk = ({"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback")
+    r = bench.roofline_of(cfg, counts, stage, pk)
+    flops = 6.0 * 4096 * 14336 * 4096
+    assert r["bound"] == "tensor" and r["achieved"] == pytest.approx(flops / 1e-3 / 1e12)
+    assert r["frac"] == pytest.approx(r["achieved"] / 1590.0)
+    dec = synth.workload("decode_bf16", T=1)
+    r = bench.roofline_of(dec, np.array([1, 1, 0, 0, 0, 0, 0, 0]), {"routed_ffn": 0.1, "shared_ffn": 0.0}, pk)
+    assert r["bound"] == "hbm"
+    assert r["achieved"] == pytest.approx(2 * 3 * 4096 * 14336 * 2 / 1e-4 / 1e9)
+    tiny = bench.roofline_of(synth.workload("tiny_f32"), np.array([64] * 8), stage, pk)
+    assert tiny["bound"] == "alu"
