@@ -51,7 +51,7 @@ Readings where the pages are silent (each also listed in the design notes):
   capacity is given, and shared experts enter with weight 1.
 * Capacity: ceil(T*k/E * factor) rows per expert ([SEV]'s script counts
   routing slots); an expert keeps its first arrivals in token order (the
-  pages say only that tokens "beyond that limit" skip the expert); a dropped
+  pages say only that the tokens past the capacity go without that expert); a dropped
   slot adds nothing and the token's other weights are not rescaled.
 * Balance loss and z-loss are computed from the bias-free router logits
   (the pages define them on the router's own output) and returned without
@@ -87,7 +87,7 @@ __all__ = [
     "quantize_rows_e4m3", "round_bf16", "e4m3_expert",
     "router_logits", "selection_key", "topk_select", "topk_gap", "softmax", "sigmoid",
     "gate_weights", "Routing", "route", "dispatch", "silu", "swiglu_expert", "moe_layer",
-    "occupancy_closed_form", "occupancy_monte_carlo", "expert_params", "moe_layer_params",
+    "combine", "occupancy_closed_form", "occupancy_monte_carlo", "expert_params", "moe_layer_params",
     "active_params",
 ]
 
@@ -231,8 +231,8 @@ def dispatch(ids: np.ndarray, n_experts: int, capacity: int | None = None):
     row_of[i]   = row of assignment i (inverse of perm), -1 when dropped
 
     With a ``capacity`` C an expert keeps its first C assignments in that
-    order and the rest skip it ([SEV]: "Tokens beyond that limit skip the
-    expert"); ``perm`` then has ``offsets[E]`` entries.
+    order and the rest skip it ([SEV]: the tokens over an expert's capacity
+    are not processed by it); ``perm`` then has ``offsets[E]`` entries.
     """
     T, k = ids.shape
     flat = ids.reshape(-1)
@@ -358,6 +358,29 @@ def moe_layer(x: np.ndarray, w_router: np.ndarray | None, bias: np.ndarray | Non
     for wts in shared_weights:
         y += ffn(x, wts)
     return y, r, w
+
+
+def combine(y_rows: np.ndarray, row_of: np.ndarray, w: np.ndarray,
+            y_shared: np.ndarray | None = None) -> np.ndarray:
+    """The weighted sum that ends the layer, from the dispatched expert rows.
+
+    [SEV] router step "Run and combine" and [TUR]'s per-expert loop: token
+    t's output is the sum over its k slots of the routing weight times the
+    output its expert produced for it, ``y[t] = sum_s w[t,s] * y_rows[row]``
+    with ``row = row_of[t*k + s]`` (the dispatch row of that assignment);
+    a dropped slot (``row = -1``) adds nothing; a shared expert's output
+    ``y_shared[t]`` is added with weight 1 ([TOK] "Shared experts").
+    """
+    w = np.asarray(w, dtype=np.float64)
+    T, k = w.shape
+    rows = np.asarray(row_of, dtype=np.int64).reshape(T, k)
+    y = np.zeros((T, y_rows.shape[1]), dtype=np.float64)
+    for s in range(k):
+        kept = rows[:, s] >= 0
+        y[kept] += w[kept, s][:, None] * np.asarray(y_rows, dtype=np.float64)[rows[kept, s]]
+    if y_shared is not None:
+        y += y_shared
+    return y
 
 
 # ---------------------------------------------------------------- 8-bit experts

@@ -332,10 +332,8 @@ def test_combine(dtype, shared):
     cfg = synth.LayerConfig("c", T, d, 8, k, 8, dtype, 0)
     moe.moe_combine(H.moe_cfg(cfg), yp, torch.from_numpy(row_of).cuda(), torch.from_numpy(w).cuda(), ys, y)
     torch.cuda.synchronize()
-    YP = H.device_to_host_f64(yp)
-    ref = np.einsum("tk,tkd->td", w.astype(np.float64), YP[row_of.reshape(T, k)])
-    if shared:
-        ref += H.device_to_host_f64(ys)
+    ref = H.oracle.combine(H.device_to_host_f64(yp), row_of, w.astype(np.float64),
+                           H.device_to_host_f64(ys) if shared else None)
     assert H.rel_err(H.device_to_host_f64(y), ref) <= (1e-6 if dtype == "f32" else 8e-3)
 
 

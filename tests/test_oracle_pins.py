@@ -674,3 +674,46 @@ def test_e4m3_expert_stays_close_to_the_float_expert(act):
         got = oracle.e4m3_expert(x, (wu, wd), act)
     err = np.max(np.abs(got - ref)) / np.max(np.abs(ref))
     assert 1e-4 < err < 0.08
+
+
+# ------------------------------------------------------------------ combine
+def test_combine_of_dispatched_rows_equals_the_per_token_sum():
+    """oracle.combine against the pages' per-token definition written with
+    plain loops here: each token adds weight x its expert's output for that
+    token (the rows sit wherever the dispatch put them), plus the shared
+    output.  Catches a transposed (t, s) index, a dropped slot that still adds,
+    or a missing shared term."""
+    rng = np.random.default_rng(11)
+    T, k, d, E = 13, 3, 5, 6
+    ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)])
+    w = rng.random((T, k))
+    _, _, perm, row_of = oracle.dispatch(ids, E, capacity=2)   # some slots dropped
+    y_rows = _rand(rng, len(perm), d)
+    ys = _rand(rng, T, d)
+    got = oracle.combine(y_rows, row_of, w, ys)
+    for t in range(T):
+        want = list(ys[t])
+        for s in range(k):
+            r = int(row_of[t * k + s])
+            if r < 0:
+                continue
+            assert perm[r] == t * k + s
+            for j in range(d):
+                want[j] += w[t, s] * y_rows[r, j]
+        assert np.allclose(got[t], want, rtol=0, atol=1e-12)
+    assert np.any(row_of < 0)
+
+
+def test_combine_of_expert_rows_reproduces_the_layer():
+    """Dispatching a small layer, running each expert on its rows and
+    combining gives the per-expert-loop layer output (both fp64)."""
+    rng = np.random.default_rng(12)
+    x, wr, wgu, wd = _layer(rng, T=11, d=6, E=5, f=4)
+    k = 2
+    y, r, w = oracle.moe_layer(x, wr, None, k, oracle.SOFTMAX_TOPK, _experts(wgu, wd), 5)
+    _, _, perm, row_of = oracle.dispatch(r.ids, 5)
+    f = wd.shape[2]
+    y_rows = np.stack([oracle.swiglu_expert(x[p // k][None], wgu[r.ids[p // k, p % k], :f],
+                                            wgu[r.ids[p // k, p % k], f:], wd[r.ids[p // k, p % k]])[0]
+                       for p in perm])
+    assert np.allclose(oracle.combine(y_rows, row_of, w), y, rtol=0, atol=1e-12)
