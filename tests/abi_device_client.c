@@ -2,7 +2,10 @@
    device memory from the CUDA runtime's C API, bf16 values as raw 16-bit
    patterns.  Built and run by tests/test_abi_c.py on a GPU; prints "ok" when
    moe_forward returns MOE_OK, the device status word is clear, every output
-   is finite and every token's gate weights sum to 1. */
+   is finite and every token's gate weights sum to 1.  With a file name as
+   its argument it also writes the layer output y (T*d bf16 bit patterns) and
+   the expert ids (T*k int32) there, for the test to compare with the oracle
+   on the same inputs (splitmix64 draws, regenerated on the Python side). */
 #include <math.h>
 #include <stdint.h>
 #include <stdio.h>
@@ -37,7 +40,7 @@ static void* upload(size_t n, float scale, uint64_t* seed) {
   return d;
 }
 
-int main(void) {
+int main(int argc, char** argv) {
   moe_config c;
   memset(&c, 0, sizeof c);
   c.T = 300;
@@ -53,14 +56,16 @@ int main(void) {
   void* wr = upload((size_t)(E * d), 0.05f, &seed);
   void* wgu = upload((size_t)(E * 2 * f * d), 0.05f, &seed);
   void* wd = upload((size_t)(E * d * f), 0.05f, &seed);
-  void *y = NULL, *w = NULL, *ws = NULL;
+  void *y = NULL, *w = NULL, *ws = NULL, *ids = NULL;
   const size_t ws_bytes = moe_workspace_bytes(&c);
   if (!x || !wr || !wgu || !wd || cudaMalloc(&y, (size_t)(T * d * 2)) != cudaSuccess ||
-      cudaMalloc(&w, (size_t)(T * k * 4)) != cudaSuccess || cudaMalloc(&ws, ws_bytes) != cudaSuccess) {
+      cudaMalloc(&w, (size_t)(T * k * 4)) != cudaSuccess || cudaMalloc(&ws, ws_bytes) != cudaSuccess ||
+      cudaMalloc(&ids, (size_t)(T * k * 4)) != cudaSuccess) {
     fprintf(stderr, "device allocation failed\n");
     return 1;
   }
-  moe_status st = moe_forward(&c, x, wr, NULL, wgu, wd, NULL, NULL, y, NULL, (float*)w, NULL, ws, ws_bytes, NULL);
+  moe_status st =
+      moe_forward(&c, x, wr, NULL, wgu, wd, NULL, NULL, y, (int32_t*)ids, (float*)w, NULL, ws, ws_bytes, NULL);
   if (st != MOE_OK) {
     fprintf(stderr, "moe_forward: %s\n", moe_status_string(st));
     return 1;
@@ -75,6 +80,16 @@ int main(void) {
   cudaMemcpy(yh, y, (size_t)(T * d * 2), cudaMemcpyDeviceToHost);
   cudaMemcpy(wh, w, (size_t)(T * k * 4), cudaMemcpyDeviceToHost);
   int bad = 0;
+  if (argc > 1) {
+    int32_t* ih = (int32_t*)malloc((size_t)(T * k * 4));
+    cudaMemcpy(ih, ids, (size_t)(T * k * 4), cudaMemcpyDeviceToHost);
+    FILE* fo = fopen(argv[1], "wb");
+    if (!fo || fwrite(yh, 2, (size_t)(T * d), fo) != (size_t)(T * d) ||
+        fwrite(ih, 4, (size_t)(T * k), fo) != (size_t)(T * k))
+      bad += 1;
+    if (fo) fclose(fo);
+    free(ih);
+  }
   for (int64_t i = 0; i < T * d; ++i) bad += (yh[i] & 0x7F80u) == 0x7F80u; /* Inf or NaN */
   for (int64_t t = 0; t < T; ++t) {
     double s = 0.0;
@@ -90,6 +105,7 @@ int main(void) {
   cudaFree(y);
   cudaFree(w);
   cudaFree(ws);
+  cudaFree(ids);
   if (bad) {
     fprintf(stderr, "%d bad values\n", bad);
     return 1;

@@ -220,8 +220,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<FP8>, 1)
             ok = false;
             break;
           }
+          // the stage's bytes from both CTAs are counted on the leader's barrier
+          if (leader) mbar_expect_tx(smem_u32(&full[stage]), 2 * (a_bytes + B_BYTES));
           const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
-          if (leader) mbar_expect_tx_cluster(fb, 2 * (a_bytes + B_BYTES));
           fill_par[stage] = (int)phase;
           tma_load_2d_pair(smem_u32(sA + stage * A_BYTES), half ? &tmA64 : &tmA, fb, kb * KB, a_row);
           if (MODE == MODE_SWIGLU) {  // 64 gate rows, then the matching 64 up rows
@@ -402,6 +403,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads<FP8>, 1)
   }
 }
 
+// Pairs that can be resident at once.  A pair needs two SMs of one GPC, and a
+// GPC with an odd number of usable SMs leaves one idle, so this can be below
+// half the SM count; a persistent grid larger than this would run its last
+// pairs' whole share of tiles after the others finish.
+template <int MODE, bool FP8>
+int resident_pairs(size_t smem, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)device_sm_count());
+  cfg.blockDim = dim3(kThreads<FP8>);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_pair_kernel<MODE, FP8>, &cfg) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    n = device_sm_count() / 2;
+  }
+  return n;
+}
+
 template <int MODE, bool FP8>
 cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& ta64, const CUtensorMap& tb, const Params& p,
                    int64_t tiles_bound, cudaStream_t stream) {
@@ -409,7 +429,7 @@ cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& ta64, const CUtenso
   cudaError_t e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<MODE, FP8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  int64_t pairs = device_sm_count() / 2;
+  int64_t pairs = resident_pairs<MODE, FP8>(smem, stream);
   if (tiles_bound < pairs) pairs = tiles_bound;
   if (pairs < 1) pairs = 1;
   grouped_gemm_pair_kernel<MODE, FP8><<<(unsigned)(2 * pairs), kThreads<FP8>, smem, stream>>>(ta, ta64, tb, p);
