@@ -89,7 +89,6 @@ struct GroupedFfnArgs {
 constexpr int kDecodeMaxCtas = 160;  // CTAs of one decode-schedule launch, at most
 constexpr int kDecodeTokens = 64;    // most tokens per unit of the decode schedule
 cudaError_t launch_grouped_ffn_bf16_tc(const GroupedFfnArgs& a, cudaStream_t stream);      // tcgen05, token rows as M
-cudaError_t launch_grouped_ffn_pair(const GroupedFfnArgs& a, cudaStream_t stream);         // tcgen05 CTA pairs, 256-row tiles
 cudaError_t launch_grouped_ffn_bf16_decode(const GroupedFfnArgs& a, cudaStream_t stream);  // tcgen05, weight rows as M
 cudaError_t launch_grouped_ffn_f32_simt(const GroupedFfnArgs& a, cudaStream_t stream);      // fp32 CUDA cores
 // decode regime: at most kDecodeTokens rows per touched group on average (uniform-routing expectation)

@@ -194,7 +194,7 @@ cudaError_t run_ffn(const moe_config* c, const Carve& k, const void* a, const in
     g.sh = shared ? k.sh_s : k.sh;
   }
   if (k.partial != nullptr && use_decode_ffn(rows, G, offsets != nullptr)) return launch_grouped_ffn_bf16_decode(g, s);
-  return launch_grouped_ffn_pair(g, s);
+  return launch_grouped_ffn_bf16_tc(g, s);
 }
 
 }  // namespace

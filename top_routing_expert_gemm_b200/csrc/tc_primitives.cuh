@@ -190,91 +190,6 @@ __device__ __forceinline__ void mma_kslice(uint32_t d_tmem, uint32_t a0, uint32_
   }
 }
 
-// ---------------------------------------------------------------- CTA pairs (cta_group::2)
-// A pair is a cluster of two CTAs on neighbouring SMs: one tcgen05.mma issued
-// by the pair's first CTA (the leader) reads A rows from both CTAs' shared
-// memory, B columns split between them, and accumulates into both CTAs'
-// tensor memory.
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// shared::cluster address of the same shared-memory offset in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-// arrive once on an mbarrier of a CTA of the cluster (this one's or the peer's)
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-// 2-D tile load into this CTA's shared memory whose completion is counted on
-// the pair leader's barrier `bar_cluster` (a shared::cluster address); no
-// multicast: each CTA loads only its own tiles
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
-                                                 int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t slot_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_smem), "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-// pair MMA: D (both CTAs' tensor memory) (+)= A (both CTAs) * B^T (split between them)
-template <bool FP8>
-__device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
-  if (FP8)
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-  else
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-// arrive once on this CTA's barrier `bar` when every pair MMA issued so far has completed
-__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-// the same arrival on the barrier at offset `bar` in both CTAs of the pair (a
-// commit signal to both CTAs' barriers; no data moves)
-__device__ __forceinline__ void mma_commit_pair_both(uint32_t bar) {
-  const uint16_t both = 0x3;
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
-               "h"(both)
-               : "memory");
-}
-// one 128-byte K slice of a stage on the pair: 4 MMAs 32 bytes apart
-template <bool FP8>
-__device__ __forceinline__ void mma_kslice_pair(uint32_t d_tmem, uint32_t a0, uint32_t b0, uint32_t idesc,
-                                                bool first) {
-#pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
-    const uint64_t ad = smem_desc_sw128(a0 + kk * 32), bd = smem_desc_sw128(b0 + kk * 32);
-    mma_pair<FP8>(d_tmem, ad, bd, idesc, (!first || kk != 0) ? 1u : 0u);
-  }
-}
-
 // Host: 2-D row-major [rows, cols] tensor map of bf16 (elem_bytes 2) or 8-bit
 // (elem_bytes 1) elements, box = box_rows x one 128-byte line, 128-byte
 // swizzle (defined in grouped_gemm_tc.cu).
