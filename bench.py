@@ -498,20 +498,33 @@ def traced_stages(layer: Layer, steps: int, flush_buf=None) -> dict:
     return out
 
 
-def roofline_of(cfg: synth.LayerConfig, counts: np.ndarray, stage: dict, peaks_: tuple) -> dict:
-    """Roofline of the grouped expert GEMMs (routed + shared), timed inside the
-    traced steps: tensor-bound large batches, HBM-bound decode-sized ones, the
-    fp32 layer on the CUDA cores."""
+def gemm_ms_in_step(stage: dict, ms_per_step: float) -> tuple[float, float]:
+    """Device time of the expert GEMMs inside a timed step: their share of the
+    traced steps (stage markers recorded between the launches) applied to the
+    timed step, so it can never exceed the step it belongs to; and the share."""
+    share = (stage["routed_ffn"] + stage["shared_ffn"]) / stage["step"]
+    return share * ms_per_step, share
+
+
+def roofline_of(cfg: synth.LayerConfig, counts: np.ndarray, stage: dict, peaks_: tuple,
+                ms_per_step: float | None = None) -> dict:
+    """Roofline of the grouped expert GEMMs (routed + shared): tensor-bound
+    large batches, HBM-bound decode-sized ones, the fp32 layer on the CUDA
+    cores.  Their time is their share of the traced steps applied to the timed
+    step (without a timed step: the traced stage time itself)."""
     pk, pk_kind = peaks_
     fl = layer_flops(cfg, counts)
     by = layer_bytes(cfg, counts)
-    g_ms = stage["routed_ffn"] + stage["shared_ffn"]
+    if ms_per_step is None:
+        g_ms, share = stage["routed_ffn"] + stage["shared_ffn"], None
+    else:
+        g_ms, share = gemm_ms_in_step(stage, ms_per_step)
     if cfg.dtype != "bf16":
         # fp32 CUDA cores: 148 SMs x 128 lanes x 2 FLOP per clock at the max SM clock
         peak = 148 * FP32_CORE_FLOP_PER_CLK_PER_SM * 1.965e9 / 1e12
         ach = (fl["experts"] + fl["shared"]) / (g_ms / 1e3) / 1e12
         return {"bound": "alu", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
-                "traffic": None, "stage_ms": g_ms,
+                "traffic": None, "stage_ms": g_ms, "share_of_step": share,
                 "kernel": "grouped_gemm_f32_kernel (CUDA cores): the two expert GEMM launches",
                 "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz"}
     if uses_decode_schedule(cfg):
@@ -531,6 +544,7 @@ def roofline_of(cfg: synth.LayerConfig, counts: np.ndarray, stage: dict, peaks_:
         r["kernel"] += " of the routed and the shared experts"
     r["traffic"] = recorded_traffic(cfg.name, "decode" if uses_decode_schedule(cfg) else "tc")
     r["stage_ms"] = g_ms
+    r["share_of_step"] = share
     return r
 
 
@@ -580,7 +594,7 @@ def measure_workload(cfg: synth.LayerConfig, steps: int, warmup: int, world: int
         "active_tflops": world * fl["total"] / (ms / 1000.0) / 1e12,
         "stage_ms": {n: stage[n] for n in STAGES},
         "traced_step_ms": stage["step"],
-        "roofline": roofline_of(cfg, counts, stage, peaks_),
+        "roofline": roofline_of(cfg, counts, stage, peaks_, ms),
         "experts_touched": int(np.sum(counts > 0)),
         "clocks": clocks,
         "l2": "flushed before every step (inputs fit in L2)" if fb is not None else

@@ -109,3 +109,14 @@ def test_roofline_of_follows_from_its_numbers():
     assert r["achieved"] == pytest.approx(2 * 3 * 4096 * 14336 * 2 / 1e-4 / 1e9)
     tiny = bench.roofline_of(synth.workload("tiny_f32"), np.array([64] * 8), stage, pk)
     assert tiny["bound"] == "alu"
+
+
+def test_gemm_time_is_its_share_of_the_traced_step_applied_to_the_timed_step():
+    stage = {"routed_ffn": 1.5, "shared_ffn": 0.5, "step": 2.5}
+    g, share = bench.gemm_ms_in_step(stage, 2.0)
+    assert share == pytest.approx(0.8) and g == pytest.approx(1.6) and g <= 2.0
+    cfg = synth.workload("mixtral_bf16")
+    pk = ({"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback")
+    r = bench.roofline_of(cfg, np.array([512] * 8), stage, pk, 2.0)
+    assert r["stage_ms"] == pytest.approx(1.6) and r["share_of_step"] == pytest.approx(0.8)
+    assert r["achieved"] == pytest.approx(6.0 * 4096 * 14336 * 4096 / 1.6e-3 / 1e12)

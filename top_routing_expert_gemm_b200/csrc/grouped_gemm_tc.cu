@@ -321,6 +321,9 @@ __global__ void __launch_bounds__(kThreads<FP8, MODE>, 1)
     const int part = (warp - 2) >> 2;                         // which of them this warp is
     const int r = q * 32 + lane;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+    // 32-byte stores when every row segment a chunk writes starts on 32
+    // bytes (the output's base is 256-byte aligned; the row pitch decides)
+    const bool st32 = (p.ldo % 16) == 0 && (reinterpret_cast<uintptr_t>(p.out) % 32) == 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t l_phase = 0;  // router: logits staged
@@ -376,9 +379,15 @@ __global__ void __launch_bounds__(kThreads<FP8, MODE>, 1)
               pk[j] = pack_bf16x2(h0, h1);
             }
             if (col_base + c + 32 <= col_lim) {
-              uint4* dst = reinterpret_cast<uint4*>(orow + c);
+              if (st32) {  // two whole 32-byte sectors
+                st_global_32B(orow + c, pk);
+                st_global_32B(orow + c + 16, pk + 8);
+              } else {
+                uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
-              for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                for (int j = 0; j < 4; ++j)
+                  dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+              }
             } else {
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
