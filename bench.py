@@ -601,7 +601,7 @@ def measure_workload(cfg: synth.LayerConfig, steps: int, warmup: int, world: int
               "not flushed: inputs larger than L2 (weights %.2f GB)" % (weight_bytes_total(cfg) / 1e9),
         "gpu_launches": steps * launches_per_step(cfg),
     }
-    if cfg.name == "decode_bf16" and rank == 0:
+    if cfg.name.startswith("decode_bf16") and rank == 0:
         rec["experts_touched_over_draws"] = decode_occupancy(layer)
     return rec, layer
 
@@ -778,6 +778,7 @@ def main() -> None:
     extra = {}
     for name, ov in parse_workloads(spec, cfg.name):
         wcfg = synth.workload(name, **ov)
+        wcfg = wcfg.replace(name=workload_key(name, ov))  # the key its DRAM-traffic record is stored under
         r, lay = measure_workload(wcfg, args.steps, args.warmup, world, rank, local, pk, flush_buf)
         extra[workload_key(name, ov)] = r
         del lay
