@@ -717,3 +717,86 @@ def test_combine_of_expert_rows_reproduces_the_layer():
                                             wgu[r.ids[p // k, p % k], f:], wd[r.ids[p // k, p % k]])[0]
                        for p in perm])
     assert np.allclose(oracle.combine(y_rows, row_of, w), y, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------------ 8-bit expert, independent evaluation
+def _e4m3_values_from_bits():
+    """Every finite E4M3 value, built here from the format's bit layout
+    (sign, four exponent bits with bias 7, three mantissa bits, exponent 0
+    subnormal, S.1111.111 reserved for NaN), with its code."""
+    out = []
+    for code in range(256):
+        e, m = (code >> 3) & 15, code & 7
+        if e == 15 and m == 7:
+            continue
+        mag = (m / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7)
+        out.append((-mag if code & 0x80 else mag, code))
+    return out
+
+
+_E4M3 = _e4m3_values_from_bits()
+
+
+def _nearest_e4m3(y: float) -> float:
+    """Exhaustive nearest E4M3 value; a tie goes to the even code (mantissa
+    LSB 0); beyond the largest value saturate."""
+    best = min(_E4M3, key=lambda vc: (abs(vc[0] - y), vc[1] & 1, vc[1]))
+    return best[0]
+
+
+def _bf16_round(v: float) -> float:
+    import struct
+    f = struct.unpack("<f", struct.pack("<f", v))[0]            # to float32, nearest even
+    b = struct.unpack("<I", struct.pack("<f", f))[0]
+    lo = b & 0xFFFF
+    b >>= 16
+    if lo > 0x8000 or (lo == 0x8000 and (b & 1)):
+        b += 1
+    return struct.unpack("<f", struct.pack("<I", (b & 0xFFFF) << 16))[0]
+
+
+def _quant_rows_python(rows):
+    """Per-row absolute-max quantisation written out: the scale and the
+    division in float32 (the precision the method decides in), then the
+    exhaustive nearest code; returns the dequantised rows."""
+    out = []
+    for row in rows:
+        r32 = [float(np.float32(v)) for v in row]
+        amax = max(abs(v) for v in r32)
+        s = float(np.float32(amax) / np.float32(448.0)) if amax > 0 else 1.0
+        out.append([_nearest_e4m3(float(np.float32(v) / np.float32(s))) * s for v in r32])
+    return out
+
+
+def _e4m3_swiglu_python(x, wg, wu, wd):
+    xd, gd, ud, dd = (_quant_rows_python(m) for m in (x, wg, wu, wd))
+    out = []
+    for xv in xd:
+        h = []
+        for j in range(len(gd)):
+            g = math.fsum(a * b for a, b in zip(xv, gd[j]))
+            u = math.fsum(a * b for a, b in zip(xv, ud[j]))
+            h.append(_bf16_round(g / (1.0 + math.exp(-g)) * u))
+        hd = _quant_rows_python([h])[0]
+        out.append([math.fsum(a * b for a, b in zip(hd, dd[i])) for i in range(len(dd))])
+    return np.array(out)
+
+
+def test_e4m3_expert_equals_a_pure_python_evaluation_of_the_scheme():
+    """oracle.e4m3_expert against the 8-bit scheme written out independently:
+    an E4M3 table from the format's bit layout, exhaustive nearest-value
+    rounding, per-row float32 scales, exact sums, h stored as bf16 and
+    re-quantised per row.  Catches a scale applied on the wrong side, a
+    missing bf16 rounding of h, a per-column instead of per-row scale, or a
+    wrong tie rule."""
+    rng = np.random.default_rng(21)
+    n, d, f = 3, 16, 8
+    x = rng.standard_normal((n, d)).astype(np.float32).astype(np.float64)
+    wg = (rng.standard_normal((f, d)) / 4).astype(np.float32).astype(np.float64)
+    wu = (rng.standard_normal((f, d)) / 4).astype(np.float32).astype(np.float64)
+    wd = (rng.standard_normal((d, f)) / 3).astype(np.float32).astype(np.float64)
+    got = oracle.e4m3_expert(x, (wg, wu, wd), oracle.ACT_SWIGLU)
+    want = _e4m3_swiglu_python(x.tolist(), wg.tolist(), wu.tolist(), wd.tolist())
+    assert np.allclose(got, want, rtol=1e-9, atol=1e-12)
+    # and it is not the float expert: quantisation moves the output
+    assert not np.allclose(got, oracle.swiglu_expert(x, wg, wu, wd), rtol=1e-4)
