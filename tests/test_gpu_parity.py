@@ -253,6 +253,7 @@ def _ragged_offsets(sizes):
     ([1, 1], 4096, 14336),                        # decode schedule: one token per expert
     ([3, 0, 40, 1], 1024, 1536),                  # decode schedule: units cut across several CTAs
     ([2100, 17, 0, 256, 257], 256, 192),          # 256-token chunks, a 9-chunk group, N = 16 remainders
+    ([300, 0, 129, 128], 448, 448),               # five-stage ring of N = 224 in both GEMMs (448 = 4 x 112 = 2 x 224)
 ])
 def test_grouped_ffn_against_dense_experts(dtype, sizes, d, f):
     rng = np.random.default_rng(sum(sizes) + d + f)
@@ -403,6 +404,7 @@ def test_quantize_e4m3_matches_the_oracle_bit_for_bit(cols):
     ([0, 1, 127, 129, 300, 0, 256], 256, 384),   # large-batch schedule
     ([3, 0, 40, 1], 1024, 1536),                  # decode schedule, units cut across CTAs
     ([600, 17], 272, 208),                        # partial weight blocks
+    ([300, 129], 480, 480),                       # partial last tile of 128 and of 256 output columns
 ])
 def test_grouped_ffn_e4m3_against_the_oracle(act, sizes, d, f):
     """8-bit experts through moe_grouped_ffn: weights quantised on the GPU,
