@@ -611,9 +611,10 @@ namespace {
 // The five-stage ring of N = 224 where it pads the output columns strictly
 // less than N = 256 (SwiGLU: 112 against 128 output columns per tile), with
 // bf16 operands, and where the group offsets fit beside it in shared memory.
-// Measured on the layer shapes: 2880 columns (12.9 tiles of 224, 11.25 of 256)
-// run 4.6% faster; where 256 divides the output the narrower tile only costs,
-// and the 8-bit kernel ran 6% slower with it.
+// Measured on the layer shapes: both GEMMs of 2880 output columns (25.7 tiles
+// of 112 against 22.5 of 128; 12.9 of 224 against 11.25 of 256) ran 2.8-4.5%
+// faster; where 256 divides the output the narrower tile only costs, and the
+// 8-bit kernel ran 6% slower with it.
 bool deep_ring(int cols, bool swiglu, bool fp8, int G) {
   if (fp8 || smem_bytes<224>(G, 0) > 227 * 1024) return false;
   const int o256 = swiglu ? 128 : 256, o224 = swiglu ? 112 : 224;
@@ -625,7 +626,9 @@ bool deep_ring(int cols, bool swiglu, bool fp8, int G) {
 template <int MODE, bool FP8>
 cudaError_t launch_ffn(bool deep, const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, int64_t tiles_bound,
                        cudaStream_t stream) {
-  if (deep) return launch_mode<MODE, 1, FP8, 224>(ta, tb, p, tiles_bound, stream);
+  if constexpr (!FP8) {
+    if (deep) return launch_mode<MODE, 1, false, 224>(ta, tb, p, tiles_bound, stream);
+  }
   return launch_mode<MODE, 1, FP8, 256>(ta, tb, p, tiles_bound, stream);
 }
 
