@@ -180,7 +180,8 @@ def test_router_topk_long_rows(gating, E, k, T, d):
     ids, w = out[0]
     H.check_routing(cfg, ids.cpu().numpy().astype(np.int64), w.cpu().numpy().astype(np.float64), r, cfg.T)
 
-@pytest.mark.parametrize("T,E,k", [(1, 1, 1), (1000, 8, 2), (4099, 256, 8), (2048, 1024, 16), (333, 5, 5)])
+@pytest.mark.parametrize("T,E,k", [(1, 1, 1), (1000, 8, 2), (4099, 256, 8), (2048, 1024, 16), (333, 5, 5),
+                                   (1024, 64, 8), (1025, 64, 8)])
 @pytest.mark.parametrize("skew", ["uniform", "one_expert", "half_empty"])
 @pytest.mark.parametrize("cf", [0.0, 1.0, 0.3])
 def test_permute_bit_exact(T, E, k, skew, cf):

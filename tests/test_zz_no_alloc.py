@@ -109,7 +109,7 @@ def test_noalloc_empty_batch_zeroes_counts_and_offsets():
     assert int(got["counts"].abs().sum()) == 0 and int(got["offsets"].abs().sum()) == 0
 
 
-@pytest.mark.parametrize("T", [40, 3000])  # single-block and count/scan/scatter paths
+@pytest.mark.parametrize("T", [40, 3000, 5000])  # one-warp, all-warp single-block and three-kernel paths
 def test_noalloc_skips_expert_ids_out_of_range_like_moe_permute(T):
     E, k, d = 8, 2, 256
     cfg = moe.make_config(T, d, E, k, 8, moe.MOE_BF16, moe.MOE_SOFTMAX_TOPK)
@@ -124,7 +124,7 @@ def test_noalloc_skips_expert_ids_out_of_range_like_moe_permute(T):
     assert int(got["offsets"][E]) == T * k - 3
 
 
-@pytest.mark.parametrize("T", [300, 5000])
+@pytest.mark.parametrize("T", [300, 2000, 5000])
 def test_noalloc_with_capacity_factor_matches_moe_permute(T):
     E, k, d = 8, 2, 128
     cfg = moe.make_config(T, d, E, k, 8, moe.MOE_BF16, moe.MOE_SOFTMAX_TOPK, capacity_factor=0.5)

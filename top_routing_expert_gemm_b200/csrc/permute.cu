@@ -251,6 +251,106 @@ __global__ void __launch_bounds__(kSmallThreads)
   }
 }
 
+// Mid-size dispatch (at most kMidDispatch assignments over at most
+// kMidExperts experts, such as a 2048-token batch with k = 2): one block as
+// well, with every warp ranking.  Warp w owns a contiguous segment of the
+// assignments and counts it per expert (__match_any_sync: one add per
+// distinct expert and round); a scan over the experts gives the offsets and
+// one over the warps each warp's first rank per expert; then each warp walks
+// its segment again in order and ranks from there.  An assignment's rank is
+// the number of earlier assignments of its expert, so the scatter is stable
+// and equal to the kernels above, in one launch instead of three.
+constexpr int64_t kMidDispatch = 8192;
+constexpr int kMidExperts = 64;
+constexpr int kMidWarps = kSmallThreads / 32;
+
+__global__ void __launch_bounds__(kSmallThreads)
+    permute_mid_kernel(const int32_t* __restrict__ ids, int64_t n, int E, int64_t capacity, int32_t* counts,
+                       int32_t* offsets, int32_t* perm, int32_t* row_of, int* status) {
+  __shared__ int wrank[kMidWarps][kMidExperts];  // per warp and expert: its count, then its first rank
+  __shared__ int base[kMidExperts];
+  __shared__ int warp_sums[kMidWarps];
+  const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+  grid_dependency_wait();  // the router's ids (programmatic launch)
+  if (tid == 0) grid_launch_dependents();
+  for (int e = lane; e < kMidExperts; e += 32) wrank[warp][e] = 0;
+  __syncwarp();
+  const int64_t seg = ((n + kMidWarps - 1) / kMidWarps + 31) / 32 * 32;  // a multiple of 32
+  const int64_t lo = (int64_t)warp * seg, hi = min(n, lo + seg);
+  const unsigned lt = (1u << lane) - 1u;
+  for (int64_t r0 = lo; r0 < hi; r0 += 32) {
+    const int64_t i = r0 + lane;
+    int e = -1;
+    if (i < hi) {
+      e = ids[i];
+      if (e < 0 || e >= E) {
+        set_status(status, kDevBadExpertId);
+        e = -1;
+      }
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) wrank[warp][e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // per expert (a thread each): the total, and each warp's first rank
+  int total = 0;
+  if (tid < E) {
+    for (int w = 0; w < kMidWarps; ++w) {
+      const int c = wrank[w][tid];
+      wrank[w][tid] = total;
+      total += c;
+    }
+  }
+  // exclusive scan of the rows each expert keeps
+  const int kept = (int)min((int64_t)total, capacity);
+  int incl = kept;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int v = warp_sums[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, v, off);
+      if (lane >= off) v += u;
+    }
+    warp_sums[lane] = v;
+  }
+  __syncthreads();
+  const int excl = incl - kept + (warp > 0 ? warp_sums[warp - 1] : 0);
+  if (tid < E) {
+    counts[tid] = total;
+    offsets[tid] = excl;
+    base[tid] = excl;
+    if (tid == E - 1) offsets[E] = excl + kept;
+  }
+  __syncthreads();
+  for (int64_t r0 = lo; r0 < hi; r0 += 32) {
+    const int64_t i = r0 + lane;
+    const bool in = i < hi;
+    int e = in ? ids[i] : -1;
+    if (e < 0 || e >= E) e = -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    int row = -1;
+    if (e >= 0) {
+      const int rank = wrank[warp][e] + __popc(peers & lt);
+      if (rank < capacity) row = base[e] + rank;
+    }
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) wrank[warp][e] += __popc(peers);
+    __syncwarp();
+    if (in) {
+      row_of[i] = row;
+      if (row >= 0) perm[row] = (int32_t)i;
+    }
+  }
+}
+
 // x_perm[row_of[t*k + s]] = x[t] for every kept slot s of token t.  Token
 // major: one warp per token reads the token's vector once (16-byte vectors,
 // four in flight per lane) and writes it to each of its rows, so x crosses
@@ -300,6 +400,11 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
     const cudaError_t e = launch_maybe_chained(permute_small_kernel, dim3(1), dim3(kSmallThreads),
                                                3 * sizeof(int) * a.E, stream, a.chained, a.ids, a.n_assign, a.E,
                                                a.capacity, a.counts, a.offsets, a.perm, a.row_of, a.status);
+    if (e != cudaSuccess) return e;
+  } else if (a.n_assign <= kMidDispatch && a.E <= kMidExperts) {
+    const cudaError_t e = launch_maybe_chained(permute_mid_kernel, dim3(1), dim3(kSmallThreads), 0, stream,
+                                               a.chained, a.ids, a.n_assign, a.E, a.capacity, a.counts, a.offsets,
+                                               a.perm, a.row_of, a.status);
     if (e != cudaSuccess) return e;
   } else {
     permute_count_kernel<<<n_chunks, kThreads, sizeof(int) * a.E, stream>>>(a.ids, a.n_assign, a.E,
