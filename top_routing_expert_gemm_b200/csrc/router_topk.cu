@@ -184,10 +184,19 @@ __global__ void __launch_bounds__(kThreads) router_topk_simt_kernel(RouterParams
     if (threadIdx.x < kWarps) z_sum[threadIdx.x] = 0.f;
     __syncthreads();
   }
-  if (W_SMEM) {
+  if (W_SMEM) {  // eight 16-byte loads in flight per thread: W_r crosses from L2 in few round trips
     const int64_t n16 = (int64_t)E * d / V;
-    for (int64_t i = threadIdx.x; i < n16; i += kThreads)
-      reinterpret_cast<uint4*>(sw)[i] = __ldg(reinterpret_cast<const uint4*>(wg) + i);
+    const uint4* src = reinterpret_cast<const uint4*>(wg);
+    uint4* dst = reinterpret_cast<uint4*>(sw);
+    int64_t i = threadIdx.x;
+    for (; i + 7 * kThreads < n16; i += 8 * kThreads) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(src + i + u * kThreads);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) dst[i + u * kThreads] = v[u];
+    }
+    for (; i < n16; i += kThreads) dst[i] = __ldg(src + i);
     __syncthreads();
   }
   const T* wsrc = W_SMEM ? sw : wg;
@@ -215,14 +224,15 @@ __global__ void __launch_bounds__(kThreads) router_topk_simt_kernel(RouterParams
           }
         }
       };
-      // four row chunks in flight per lane: the x row streams from HBM
+      // eight row chunks in flight per lane: the x row streams from HBM
+      // (with a token or two per warp the row's latency is the cost)
       int i0 = lane * V;
-      for (; i0 + 3 * 32 * V < d; i0 += 4 * 32 * V) {
-        Vec16<T> xv[4];
+      for (; i0 + 7 * 32 * V < d; i0 += 8 * 32 * V) {
+        Vec16<T> xv[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) xv[u] = ld16(xr + i0 + u * 32 * V);
+        for (int u = 0; u < 8; ++u) xv[u] = ld16(xr + i0 + u * 32 * V);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) fma_chunk(xv[u], i0 + u * 32 * V);
+        for (int u = 0; u < 8; ++u) fma_chunk(xv[u], i0 + u * 32 * V);
       }
       for (; i0 < d; i0 += 32 * V) fma_chunk(ld16(xr + i0), i0);
 #pragma unroll
