@@ -616,7 +616,7 @@ namespace {
 // faster; where 256 divides the output the narrower tile only costs, and the
 // 8-bit kernel ran 6% slower with it.
 bool deep_ring(int cols, bool swiglu, bool fp8, int G) {
-  if (fp8 || smem_bytes<224>(G, 0) > 227 * 1024) return false;
+  if (fp8 || smem_bytes<224>(G, 0) > (size_t)device_smem_per_block()) return false;
   const int o256 = swiglu ? 128 : 256, o224 = swiglu ? 112 : 224;
   const int64_t pad256 = (int64_t)((cols + o256 - 1) / o256) * o256 - cols;
   const int64_t pad224 = (int64_t)((cols + o224 - 1) / o224) * o224 - cols;

@@ -121,5 +121,6 @@ struct CombineArgs {
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
 
 int device_sm_count();
+int device_smem_per_block();  // opt-in dynamic shared memory per block (227 KiB on B200)
 
 }  // namespace moe

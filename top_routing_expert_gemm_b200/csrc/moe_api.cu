@@ -20,6 +20,14 @@ int device_sm_count() {
   return n;
 }
 
+int device_smem_per_block() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 227 * 1024;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess || n <= 0)
+    return 227 * 1024;
+  return n;
+}
+
 // Router kernel choice: with many experts the router is a real GEMM
 // (2*T*d*E flops: 30 GFLOP for T=8192, d=7168, E=256) and runs on the tensor
 // cores with the top-k fused into the epilogue; with few experts (or fp32,
