@@ -101,12 +101,14 @@ def replica_throughput(tokens_per_rank: int, world: int, ms_max: float) -> float
 
 def launches_per_step(cfg) -> int:
     """Kernels of ours one moe_forward step launches: router, dispatch (one
-    block-wide kernel for at most 1024 assignments, else count / scan /
-    scatter) and the row gather (with 8-bit experts the gather-quantise), two
-    expert GEMMs for the routed experts (8-bit: with the re-quantisation of h
-    between them) and for each shared expert (8-bit: after quantising x, and
-    with the re-quantisation of h), and the combine."""
-    dispatch = 2 if cfg.T * cfg.top_k <= 1024 else 4
+    block-wide kernel for at most 1024 assignments, or at most 8192 over at
+    most 64 experts, else count / scan / scatter) and the row gather (with
+    8-bit experts the gather-quantise), two expert GEMMs for the routed
+    experts (8-bit: with the re-quantisation of h between them) and for each
+    shared expert (8-bit: after quantising x, and with the re-quantisation of
+    h), and the combine."""
+    n = cfg.T * cfg.top_k
+    dispatch = 2 if n <= 1024 or (n <= 8192 and cfg.n_experts <= 64) else 4
     routed = 2 + (1 if cfg.e4m3 else 0)
     shared = cfg.n_shared * (2 + (2 if cfg.e4m3 else 0))
     return 1 + dispatch + routed + shared + 1

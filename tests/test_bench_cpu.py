@@ -57,14 +57,15 @@ def test_layer_flops_and_bytes():
 
 
 def test_launches_per_step():
-    assert bench.launches_per_step(synth.workload("mixtral_bf16")) == 8
+    assert bench.launches_per_step(synth.workload("mixtral_bf16")) == 6   # 4096 assignments, 8 experts: one-block sort
     assert bench.launches_per_step(synth.workload("decode_bf16", T=1)) == 6
     assert bench.launches_per_step(synth.workload("deepseek_bf16")) == 10
     assert bench.launches_per_step(synth.workload("tiny_f32")) == 6   # one-block sort, gather, 2 GEMMs
     # 8-bit: gather-quantise in place of the gather, h re-quantised between the
     # routed GEMMs, the shared expert's x and h quantised
-    assert bench.launches_per_step(synth.workload("mixtral_bf16", e4m3=True)) == 9
+    assert bench.launches_per_step(synth.workload("mixtral_bf16", e4m3=True)) == 7
     assert bench.launches_per_step(synth.workload("deepseek_bf16", e4m3=True)) == 13
+    assert bench.launches_per_step(synth.workload("gptoss_bf16")) == 8    # 32768 assignments: count / scan / scatter
 
 
 def test_workload_keys_and_selection():
