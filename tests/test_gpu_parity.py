@@ -498,3 +498,45 @@ def test_forward_bf16_equals_the_stage_calls(cfg):
     assert out["status"] == 0
     y = _stage_by_stage(inp)
     assert torch.equal(out["y"].view(torch.int16), y.view(torch.int16))
+
+
+@pytest.mark.parametrize("cfg", [
+    SMALL["mixtral_like"],
+    SMALL["deepseek_like"],                                       # shared expert: six stages all non-empty
+    synth.LayerConfig("decode_traced", 4, 512, 8, 2, 1024, "bf16", synth.SOFTMAX_TOPK, seed=43),
+], ids=lambda c: c.name)
+def test_forward_traced_equals_forward_and_records_its_stages(cfg):
+    """moe_forward_traced runs the same launches as moe_forward with six
+    events recorded between them: bitwise the same outputs, every event
+    recorded on the launching stream, in order, and the stage times add up to
+    the step's."""
+    inp = H.make_inputs(cfg)
+    ref = H.run_forward(inp)
+    assert ref["status"] == 0
+    c = H.moe_cfg(cfg)
+    dev = inp.dev
+    T, k, E, d = cfg.T, cfg.top_k, cfg.n_experts, cfg.d_model
+    y = torch.empty(T, d, dtype=H.torch_dtype(cfg), device="cuda")
+    ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    ws = torch.empty(max(256, moe.moe_workspace_bytes(c)), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.Stream()                                  # not the current stream
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    moe.moe_forward_traced(c, dev["x"], dev["w_router"], dev["bias"], dev["w_gate_up"], dev["w_down"],
+                           dev.get("ws_gate_up"), dev.get("ws_down"), y, ids, w, counts, ws, stream=stream,
+                           stage_events=evs)
+    assert moe.moe_device_status(ws, stream=stream) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), ref["y"].view(torch.int16))
+    assert torch.equal(ids, ref["ids"]) and torch.equal(w, ref["w"]) and torch.equal(counts, ref["counts"])
+    assert all(e.query() for e in evs)
+    stages = [evs[j].elapsed_time(evs[j + 1]) for j in range(5)]
+    assert all(s >= 0.0 for s in stages)
+    assert abs(sum(stages) - evs[0].elapsed_time(evs[5])) <= 1e-3 + 1e-3 * evs[0].elapsed_time(evs[5])
+    # None entries are skipped
+    moe.moe_forward_traced(c, dev["x"], dev["w_router"], dev["bias"], dev["w_gate_up"], dev["w_down"],
+                           dev.get("ws_gate_up"), dev.get("ws_down"), y, ids, w, counts, ws, stream=stream,
+                           stage_events=[evs[0], None, None, None, None, evs[5]])
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), ref["y"].view(torch.int16))
