@@ -61,10 +61,10 @@ __device__ __forceinline__ float row_scale(float amax) {
 
 // Row r of src -> codes row r and scale[r]; rows past *rows_dev (when given)
 // are left alone.  A pass for the absolute maximum, then a pass that converts
-// (it finds the row in L1).  Four independent 16-byte loads in flight per
-// lane; 40 registers, so that many warps per SM hide the latency of the loads
-// and of the IEEE divisions (a variant holding the whole row in registers ran
-// at one block per SM and measured slower).
+// (it finds the row in L1).  Eight independent 16-byte loads in flight per
+// lane, with registers left for many warps per SM to hide the latency of the
+// loads and of the IEEE divisions (a variant holding the whole row in
+// registers ran at one block per SM and measured slower).
 __global__ void __launch_bounds__(kThreads)
     quantize_rows_e4m3_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, const int32_t* rows_dev,
                               int cols, uint8_t* __restrict__ q, float* __restrict__ scale) {
@@ -76,20 +76,23 @@ __global__ void __launch_bounds__(kThreads)
     const uint4* row = reinterpret_cast<const uint4*>(src + r * cols);
     float amax = 0.f;
     int v = lane;
-    for (; v + 96 < nv; v += 128) {  // four independent loads in flight per lane
-      const uint4 a0 = __ldg(row + v), a1 = __ldg(row + v + 32), a2 = __ldg(row + v + 64), a3 = __ldg(row + v + 96);
-      amax = amax8(a3, amax8(a2, amax8(a1, amax8(a0, amax))));
+    for (; v + 7 * 32 < nv; v += 8 * 32) {  // eight independent loads in flight per lane
+      uint4 a[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a[i] = __ldg(row + v + 32 * i);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = amax8(a[i], amax);
     }
     for (; v < nv; v += 32) amax = amax8(__ldg(row + v), amax);
     const float s = row_scale(amax);
     if (lane == 0) scale[r] = s;
     uint2* out = reinterpret_cast<uint2*>(q + r * cols);
-    for (v = lane; v + 96 < nv; v += 128) {
-      const uint4 a0 = __ldg(row + v), a1 = __ldg(row + v + 32), a2 = __ldg(row + v + 64), a3 = __ldg(row + v + 96);
-      out[v] = e4m3x8(a0, s);
-      out[v + 32] = e4m3x8(a1, s);
-      out[v + 64] = e4m3x8(a2, s);
-      out[v + 96] = e4m3x8(a3, s);
+    for (v = lane; v + 7 * 32 < nv; v += 8 * 32) {
+      uint4 a[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a[i] = __ldg(row + v + 32 * i);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) out[v + 32 * i] = e4m3x8(a[i], s);
     }
     for (; v < nv; v += 32) out[v] = e4m3x8(__ldg(row + v), s);
   }
