@@ -126,6 +126,9 @@ struct Params {
   int32_t* ids;            // [rows, k]
   float* wts;              // [rows, k]
   int E, k, gating, bias_select_only;
+  // 8-bit GEMM-1 only: per row, the largest |h| stored, as bf16 bits (an
+  // atomic maximum over the row's tiles; zero on entry), or null
+  uint32_t* row_amax;
 };
 
 // router: the tile's logits are staged in shared memory over the drained
@@ -356,6 +359,8 @@ __global__ void __launch_bounds__(kThreads<FP8, MODE>, 1)
       if (MODE != MODE_ROUTER) {
         // SwiGLU mode: gate in accumulator columns [0, bno), up in [bno, 2 bno);
         // plain mode: the bno output columns
+        constexpr bool kRowMax = FP8 && (MODE == MODE_SWIGLU || MODE == MODE_GELU);
+        uint32_t amax_bits = 0;  // kRowMax: the largest |h| this thread stores, as bf16 bits
 #pragma unroll 1
         for (int c = 32 * part; c < bno; c += 32 * kPerQuarter) {
           uint32_t v[32], u[32];
@@ -388,6 +393,14 @@ __global__ void __launch_bounds__(kThreads<FP8, MODE>, 1)
               }
               pk[j] = pack_bf16x2(h0, h1);
             }
+            if (kRowMax && p.row_amax) {  // over the stored columns, as the re-quantisation reads them
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const int cc = col_base + c + 2 * j;
+                if (cc < col_lim) amax_bits = max(amax_bits, pk[j] & 0x7FFFu);
+                if (cc + 1 < col_lim) amax_bits = max(amax_bits, (pk[j] >> 16) & 0x7FFFu);
+              }
+            }
             if (col_base + c + 32 <= col_lim) {
               if (st32) {  // two whole 32-byte sectors
                 st_global_32B(orow + c, pk);
@@ -414,6 +427,7 @@ __global__ void __launch_bounds__(kThreads<FP8, MODE>, 1)
             }
           }
         }
+        if (kRowMax && p.row_amax && ok && amax_bits) atomicMax(p.row_amax + grow, amax_bits);
       } else {
         // Router: keep the top k of kappa = logit + bias over the E columns of
         // each row, then the gate weights of the chosen experts.  The CTA owns
@@ -651,12 +665,20 @@ cudaError_t run_tc(const GroupedFfnArgs& a, cudaStream_t stream) {
                         : nullptr;
   CUtensorMap mA1, mB1;
   cudaError_t e;
+  // 8-bit: GEMM-1's epilogue leaves each row's largest |h| in sh (as bf16
+  // bits), so the re-quantisation of h reads h once
+  uint32_t* row_amax = FP8 ? reinterpret_cast<uint32_t*>(a.sh) : nullptr;
+  if (FP8) {
+    e = cudaMemsetAsync(a.sh, 0, sizeof(float) * (size_t)a.rows, stream);
+    if (e != cudaSuccess) return e;
+  }
   if (gelu) {
     // GEMM-1 + GELU: tile = 128 rows x n1 up columns
     if (!make_map(&mA1, a.a, a.rows, a.d, BM, eb) || !make_map(&mB1, a.w_gate_up, w1_rows, a.d, n1, eb))
       return cudaErrorInvalidValue;
     Params p1{a.offsets, G, a.rows, a.d, a.f, (a.f + n1 - 1) / n1, (int64_t)a.f, 0, a.h, a.f, a.status, lim, n1,
               a.sa, s1};
+    p1.row_amax = row_amax;
     e = launch_ffn<MODE_GELU, FP8>(deep1, mA1, mB1, p1, mt_bound * p1.nt, stream);
   } else {
     // GEMM-1 + SwiGLU: tile = 128 rows x (n1/2 gate + n1/2 up) columns
@@ -664,13 +686,15 @@ cudaError_t run_tc(const GroupedFfnArgs& a, cudaStream_t stream) {
       return cudaErrorInvalidValue;
     Params p1{a.offsets, G, a.rows, a.d, a.f, (a.f + n1 / 2 - 1) / (n1 / 2), 2 * (int64_t)a.f, a.f, a.h, a.f,
               a.status, lim, n1, a.sa, s1};
+    p1.row_amax = row_amax;
     e = launch_ffn<MODE_SWIGLU, FP8>(deep1, mA1, mB1, p1, mt_bound * p1.nt, stream);
   }
   if (e != cudaSuccess) return e;
   const void* a2 = a.h;
   const float* sa2 = nullptr;
   if (FP8) {  // h -> E4M3 codes and per-token scales
-    e = launch_quantize_e4m3(a.h, a.rows, a.offsets ? a.offsets + a.G : nullptr, a.f, a.hq, a.sh, stream);
+    e = launch_quantize_e4m3(a.h, a.rows, a.offsets ? a.offsets + a.G : nullptr, a.f, a.hq, a.sh, stream,
+                             row_amax);
     if (e != cudaSuccess) return e;
     a2 = a.hq;
     sa2 = a.sh;

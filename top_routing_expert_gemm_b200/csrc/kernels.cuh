@@ -97,9 +97,11 @@ int64_t decode_partial_slots();  // [128][64] fp32 tiles
 int64_t decode_counter_cap(int64_t rows, int G, int d, int f);
 
 // ---- FP8 E4M3 row quantisation (quant_e4m3.cu): per row s = max|x| / 448,
-// q = e4m3(x / s); rows past *rows_dev (when given) are left alone
+// q = e4m3(x / s); rows past *rows_dev (when given) are left alone.
+// amax_bits (may be `scale` itself): each row's max|x| as bf16 bits, known
+// ahead, so the row is read once
 cudaError_t launch_quantize_e4m3(const void* src, int64_t rows, const int32_t* rows_dev, int cols, uint8_t* q,
-                                 float* scale, cudaStream_t stream);
+                                 float* scale, cudaStream_t stream, const uint32_t* amax_bits = nullptr);
 // the dispatch with 8-bit experts: token t of x [T, cols] quantised once, its
 // codes and scale written to every kept row row_of[t*k + s]
 cudaError_t launch_gather_quantize_e4m3(const void* x, const int32_t* row_of, int k, int64_t T, int cols,

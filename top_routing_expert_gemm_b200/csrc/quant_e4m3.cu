@@ -60,31 +60,39 @@ __device__ __forceinline__ float row_scale(float amax) {
 }
 
 // Row r of src -> codes row r and scale[r]; rows past *rows_dev (when given)
-// are left alone.  A pass for the absolute maximum, then a pass that converts
+// are left alone.  A pass for the absolute maximum (skipped when amax_bits
+// holds it: the 8-bit GEMM-1 leaves it there for h), then a pass that converts
 // (it finds the row in L1).  Eight independent 16-byte loads in flight per
 // lane, with registers left for many warps per SM to hide the latency of the
 // loads and of the IEEE divisions (a variant holding the whole row in
 // registers ran at one block per SM and measured slower).
 __global__ void __launch_bounds__(kThreads)
     quantize_rows_e4m3_kernel(const __nv_bfloat16* __restrict__ src, int64_t rows, const int32_t* rows_dev,
-                              int cols, uint8_t* __restrict__ q, float* __restrict__ scale) {
+                              int cols, uint8_t* __restrict__ q, float* scale, const uint32_t* amax_bits) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t dr = rows_dev ? (int64_t)*rows_dev : rows;
   const int64_t n = dr < rows ? dr : rows;
   const int nv = cols / 8;
   for (int64_t r = (int64_t)blockIdx.x * kWarps + warp; r < n; r += (int64_t)gridDim.x * kWarps) {
     const uint4* row = reinterpret_cast<const uint4*>(src + r * cols);
-    float amax = 0.f;
+    float s;
     int v = lane;
-    for (; v + 7 * 32 < nv; v += 8 * 32) {  // eight independent loads in flight per lane
-      uint4 a[8];
+    if (amax_bits) {  // the row's maximum is known: read it before its scale overwrites it
+      const float amax = __uint_as_float(amax_bits[r] << 16);
+      s = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+      __syncwarp();
+    } else {
+      float amax = 0.f;
+      for (; v + 7 * 32 < nv; v += 8 * 32) {  // eight independent loads in flight per lane
+        uint4 a[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) a[i] = __ldg(row + v + 32 * i);
+        for (int i = 0; i < 8; ++i) a[i] = __ldg(row + v + 32 * i);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = amax8(a[i], amax);
+        for (int i = 0; i < 8; ++i) amax = amax8(a[i], amax);
+      }
+      for (; v < nv; v += 32) amax = amax8(__ldg(row + v), amax);
+      s = row_scale(amax);
     }
-    for (; v < nv; v += 32) amax = amax8(__ldg(row + v), amax);
-    const float s = row_scale(amax);
     if (lane == 0) scale[r] = s;
     uint2* out = reinterpret_cast<uint2*>(q + r * cols);
     for (v = lane; v + 7 * 32 < nv; v += 8 * 32) {
@@ -147,10 +155,10 @@ int64_t grid_for(int64_t units) {
 }  // namespace
 
 cudaError_t launch_quantize_e4m3(const void* src, int64_t rows, const int32_t* rows_dev, int cols, uint8_t* q,
-                                 float* scale, cudaStream_t stream) {
+                                 float* scale, cudaStream_t stream, const uint32_t* amax_bits) {
   if (rows == 0) return cudaSuccess;
   quantize_rows_e4m3_kernel<<<(unsigned)grid_for(rows), kThreads, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(src), rows, rows_dev, cols, q, scale);
+      static_cast<const __nv_bfloat16*>(src), rows, rows_dev, cols, q, scale, amax_bits);
   return cudaGetLastError();
 }
 
