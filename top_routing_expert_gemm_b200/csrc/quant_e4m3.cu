@@ -121,9 +121,12 @@ __global__ void __launch_bounds__(kThreads)
     const int my_row = lane < k ? row_of[t * k + lane] : -1;  // k <= kMaxTopK <= 32
     float amax = 0.f;
     int v = lane;
-    for (; v + 96 < nv; v += 128) {
-      const uint4 a0 = __ldg(row + v), a1 = __ldg(row + v + 32), a2 = __ldg(row + v + 64), a3 = __ldg(row + v + 96);
-      amax = amax8(a3, amax8(a2, amax8(a1, amax8(a0, amax))));
+    for (; v + 7 * 32 < nv; v += 8 * 32) {  // eight independent loads in flight per lane
+      uint4 a[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a[i] = __ldg(row + v + 32 * i);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = amax8(a[i], amax);
     }
     for (; v < nv; v += 32) amax = amax8(__ldg(row + v), amax);
     const float s = row_scale(amax);
